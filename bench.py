@@ -1,0 +1,486 @@
+#!/usr/bin/env python
+"""Benchmark: MoE layer forward (route + pack + compute + combine) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Default workload: the Granite-shaped stack (T=1412, d=1024, E=32, top-8, SwiGLU d_ff=512,
+24 layers chained by the residual, bf16).  A step is one forward of the whole stack.  The
+metric is routed tokens per second per MoE layer forward: T * layers / step time, summed
+over ranks.  With N > 1 each rank runs an independent replica of the workload (weak
+scaling, no collective on the data path).  Prints one JSON line (rank 0).
+
+--impl reference times the fp64 CPU oracle on the host cores (a bounded sample per step).
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "routed tokens/s per MoE layer fwd (1×B200) + % of bf16 TC / HBM roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS = ["route", "pack", "gemm_gate_up", "gemm_down", "combine"]
+KERNEL_SOURCES = {"route": ["route.cu"], "pack": ["dispatch.cu"],
+                  "gemm_gate_up": ["gemm_sm100.cu", "common.cuh"],
+                  "gemm_down": ["gemm_sm100.cu", "common.cuh"], "combine": ["combine.cu"]}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="granite24")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--profiled-steps", type=int, default=20,
+                    help="timed steps that also record per-kernel events")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true", help="replay the step as a CUDA graph")
+    a = ap.parse_args()
+    a.warmup = max(a.warmup, 3)
+    return a
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    Q = ("timestamp,index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,"
+         "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id=None):
+        self.proc = None
+        self.bus_id = bus_id
+        self.path = tempfile.mktemp(suffix=".csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv",
+                                          "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for r in csv.reader(f):
+                if len(r) < 11 or r[0].startswith("timestamp"):
+                    continue
+                r = [c.strip() for c in r]
+                try:
+                    ts = time.mktime(time.strptime(r[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    ts += float("0." + r[0].split(".")[1]) if "." in r[0] else 0.0
+                except ValueError:
+                    continue
+                rows.append((ts, r))
+        os.unlink(self.path)
+        if self.bus_id:
+            sel = [x for x in rows if x[1][2].lower().endswith(self.bus_id.lower()[-12:])]
+            rows = sel or rows
+        inside = [x for x in rows if t0 - 0.1 <= x[0] <= t1 + 0.1] or rows
+        if not inside:
+            return None
+        mhz = [float(r[3].split()[0]) for _, r in inside if r[3].split()[0].replace(".", "").isdigit()]
+        mx = [float(r[4].split()[0]) for _, r in inside if r[4].split()[0].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for _, r in inside for n, v in zip(names, r[7:11]) if v == "Active"})
+        return {"sm_mhz": statistics.median(mhz) if mhz else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(inside)}
+
+
+# ----------------------------------------------------------------------------- cost model
+
+def kernel_costs(wl, R, touched):
+    """Algorithmic bytes and flops per launch of each kernel for one layer.
+
+    R: kept routed rows; touched: experts with at least one kept row."""
+    esz = 2 if wl.dtype == "bf16" else 4
+    T, d, E, k, F = wl.T, wl.d, wl.E, wl.k, wl.d_ff
+    sh = 1 if wl.has_shared else 0
+    Rp = R + sh * T                     # rows through the expert GEMMs
+    nw = touched + sh                   # weight sets streamed
+    c = {}
+    c["route"] = dict(bytes=T * d * esz + E * d * esz + T * k * 8 + E * 4, flops=2.0 * T * d * E)
+    c["pack"] = dict(bytes=T * d * esz + R * d * esz + T * k * 8 + R * 4, flops=0.0)
+    c["gemm_gate_up"] = dict(bytes=nw * 2 * F * d * esz + Rp * d * esz + Rp * F * esz,
+                             flops=4.0 * Rp * d * F)
+    c["gemm_down"] = dict(bytes=nw * d * F * esz + Rp * F * esz + Rp * d * esz,
+                          flops=2.0 * Rp * d * F)
+    c["combine"] = dict(bytes=R * d * esz + T * d * esz * (1 + int(wl.add_residual) + sh) + T * k * 8,
+                        flops=0.0)
+    return c
+
+
+def traffic_from_profiles(kernel, workload):
+    """ncu DRAM bytes per launch recorded under profiles/, if the kernel source is unchanged."""
+    pdir = os.path.join(ROOT, "profiles")
+    srcdir = os.path.join(ROOT, "routing_dispatch_expert_gemm_b200", "csrc")
+    h = hashlib.sha1()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(srcdir, f), "rb") as fh:
+            h.update(fh.read())
+    sha = h.hexdigest()[:12]
+    if not os.path.isdir(pdir):
+        return None
+    pat = re.compile(r"traffic_bytes_per_launch\s+%s@%s\s*=\s*([0-9.eE+]+)\s+sources\s+([0-9a-f]+)"
+                     % (re.escape(kernel), re.escape(workload)))
+    for fn in sorted(os.listdir(pdir)):
+        if not fn.endswith((".md", ".txt")):
+            continue
+        with open(os.path.join(pdir, fn)) as f:
+            for line in f:
+                m = pat.search(line)
+                if m and m.group(2) == sha:
+                    return float(m.group(1))
+    return None
+
+
+def source_sha(kernel):
+    srcdir = os.path.join(ROOT, "routing_dispatch_expert_gemm_b200", "csrc")
+    h = hashlib.sha1()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(srcdir, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_sample_rate(wl, x, layers, budget_s=12.0, max_layers=None, n_tokens=None, seed=0):
+    """Time the oracle as it stands on a bounded sample; returns (tokens*layers/s, sample, s).
+
+    Routing and the capacity pass always cover all T tokens; the expert FFN and combine run
+    for all tokens, or for a seeded sample of ``n_tokens`` (default: all tokens when the
+    layer is small, 32 when it is large)."""
+    import numpy as np
+
+    from oracle import moe_oracle as O
+    C = None if wl.phi is None else O.capacity(wl.T, wl.k, wl.E, *wl.phi)
+    if n_tokens is None and wl.T * wl.k * wl.d * wl.d_ff > 4e10:
+        n_tokens = 32
+    toks = None
+    if n_tokens is not None and n_tokens < wl.T:
+        toks = np.sort(np.random.default_rng(seed).choice(wl.T, size=n_tokens, replace=False))
+    t0 = time.perf_counter()
+    done = 0
+    xin = x
+    for p in layers:
+        y, _ = O.moe_layer(xin, p, wl.k, wl.gate_mode, C, add_residual=wl.add_residual, tokens=toks)
+        done += 1
+        if wl.add_residual and toks is None:
+            xin = O.round_to_bf16(y) if wl.dtype == "bf16" else y
+        if time.perf_counter() - t0 > budget_s or (max_layers and done >= max_layers):
+            break
+    el = time.perf_counter() - t0
+    ntok = wl.T if toks is None else len(toks)
+    sample = (f"{done} of {len(layers)} layers x {ntok} of {wl.T} tokens "
+              f"(routing and capacity over all tokens), fp64 numpy")
+    return ntok * done / el, sample, el
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(a):
+    import torch
+    import torch.distributed as dist
+
+    from routing_dispatch_expert_gemm_b200 import build, inputs as I, native as N
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    N.lib()
+
+    wl = I.WORKLOADS[a.workload]
+    L = wl.layers
+    x, layers = I.make_inputs(wl, seed=a.seed + rank, device=dev)
+    cap = -1 if wl.phi is None else N.moe_capacity(wl.T, wl.k, wl.E, *wl.phi)
+    cfg = N.make_config(wl.T, wl.d, wl.E, wl.k, wl.d_ff, dtype=wl.dtype, gate_mode=wl.gate_mode,
+                        capacity=cap, has_shared=wl.has_shared, add_residual=wl.add_residual)
+    ws = N.workspace(cfg, dev)
+    ybuf = [torch.empty_like(x), torch.empty_like(x)]
+    demand = torch.zeros((L, wl.E), dtype=torch.int32, device=dev)
+    offsets = torch.zeros((L, wl.E + 2), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(xin, evs=None):
+        h = xin
+        for l, p in enumerate(layers):
+            y = ybuf[l % 2]
+            args = (cfg, h, p["w_router"], p["logit_bias"], p["w_gate"], p["w_up"], p["w_down"],
+                    p["shared_gate"], p["shared_up"], p["shared_down"], y, None, None,
+                    demand[l], offsets[l])
+            if evs is None:
+                N.moe_forward(*args, ws, stream)
+            else:
+                N.moe_forward_profiled(*args, evs[l], ws, stream)
+            h = y
+        return h
+
+    # weights + activations per step vs L2: flush only when the step fits in L2
+    step_bytes = sum(t.numel() * t.element_size() for p in layers for t in p.values()
+                     if t is not None)
+    flush = None
+    if step_bytes < 256e6:
+        flush = torch.empty(int(512e6) // 4, dtype=torch.int32, device=dev)
+
+    for _ in range(a.warmup):
+        step(x)
+    torch.cuda.synchronize(dev)
+    st = N.moe_get_device_status(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    nprof = min(a.profiled_steps, a.steps)
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(L)]
+           for _ in range(nprof)]
+    for s in evs:  # create the handles before timing
+        for l in s:
+            for e in l:
+                e.record(stream)
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(a.steps)]
+    bus = None
+    try:
+        pr = torch.cuda.get_device_properties(dev)
+        bus = "%02X:%02X.0" % (pr.pci_bus_id, pr.pci_device_id)
+    except Exception:
+        pass
+    clocks = ClockSampler(bus)
+    clocks.start()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t0 = time.time()
+    for s in range(a.steps):
+        if flush is not None:
+            flush.zero_()
+        step_ev[s][0].record(stream)
+        step(x, evs[s] if s < nprof else None)
+        step_ev[s][1].record(stream)
+    torch.cuda.synchronize(dev)
+    t1 = time.time()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop(t0, t1)
+    ms_total = sum(b.elapsed_time(e) for b, e in step_ev)
+    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total = float(t.item())
+    ms_per_step = ms_total / a.steps
+    value = world * wl.T * L / (ms_per_step / 1e3)
+    st = N.moe_get_device_status(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after timing")
+
+    # per-kernel live timings
+    per = {k: [] for k in KERNELS}
+    for s in range(nprof):
+        for l in range(L):
+            e = evs[s][l]
+            for i, kname in enumerate(KERNELS):
+                per[kname].append(e[i].elapsed_time(e[i + 1]))
+    avg_ms = {k: statistics.mean(v) for k, v in per.items()}
+    tot_ms = {k: sum(v) for k, v in per.items()}
+    dom = max(tot_ms, key=tot_ms.get)
+
+    dem = demand.cpu()
+    offs = offsets.cpu()
+    Rs = [int(offs[l, wl.E]) for l in range(L)]
+    touched = [int((offs[l, 1:wl.E + 1] - offs[l, :wl.E] > 0).sum()) for l in range(L)]
+    costs = [kernel_costs(wl, R, tc) for R, tc in zip(Rs, touched)]
+    peaks, peak_src = load_peaks()
+    pk_tc = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    pk_hbm = peaks["hbm_gbs"]
+
+    def roof(kname):
+        b = statistics.mean(c[kname]["bytes"] for c in costs)
+        fl = statistics.mean(c[kname]["flops"] for c in costs)
+        t_s = avg_ms[kname] / 1e3
+        t_tc = fl / (pk_tc * 1e12)
+        t_hbm = b / (pk_hbm * 1e9)
+        if t_tc >= t_hbm:
+            ach = fl / t_s / 1e12
+            r = {"bound": "tensor", "achieved": ach, "peak": pk_tc, "unit": "TFLOP/s",
+                 "frac": ach / pk_tc}
+        else:
+            ach = b / t_s / 1e9
+            r = {"bound": "hbm", "achieved": ach, "peak": pk_hbm, "unit": "GB/s",
+                 "frac": ach / pk_hbm}
+        r.update(kernel=kname, algorithmic_bytes=b, algorithmic_flops=fl,
+                 avg_launch_us=avg_ms[kname] * 1e3, peak_source=peak_src)
+        return r
+
+    roofline = roof(dom)
+    roofline["traffic"] = traffic_from_profiles(dom, wl.name)
+    roofline["source_sha"] = source_sha(dom)
+    breakdown = {k: {"avg_us": round(avg_ms[k] * 1e3, 2), "share": round(tot_ms[k] / sum(tot_ms.values()), 4),
+                     "frac": round(roof(k)["frac"], 4), "bound": roof(k)["bound"]} for k in KERNELS}
+
+    # end to end through the public API: pinned host x in, pinned host y out, every step
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty_like(x_host).pin_memory()
+    x_dev = torch.empty_like(x)
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        y_host.copy_(step(x_dev), non_blocking=True)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(a.steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        y_host.copy_(step(x_dev), non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item()) / a.steps
+    nbytes = x.numel() * x.element_size()
+    e2e = {"value": world * wl.T * L / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
+           "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes}
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        xs = x.cpu()
+        lc = [{k: (v.cpu() if v is not None else None) for k, v in p.items()} for p in layers]
+        rate, sample, el = oracle_sample_rate(wl, xs, lc)
+        cpu = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": sample, "seconds": round(el, 2)}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k,
+                   "d_ff": wl.d_ff, "layers": L, "gate_mode": wl.gate_mode,
+                   "capacity": cap, "shared_expert": wl.has_shared,
+                   "residual": wl.add_residual, "parallelism": f"replicas{world}",
+                   "l2": ("flushed between steps" if flush is not None else
+                          f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB of weights per step)")},
+        "roofline": roofline, "kernels": breakdown, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": a.steps * L * 5, "clocks": clk,
+        "routes_per_step": int(dem.sum()),
+    }
+    print(json.dumps(out), flush=True)
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import torch
+
+    from routing_dispatch_expert_gemm_b200 import inputs as I
+
+    wl = I.WORKLOADS[a.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    x, layers = I.make_inputs(wl, seed=a.seed, device=dev, layers=1)
+    xs = x.cpu()
+    lc = [{k: (v.cpu() if v is not None else None) for k, v in p.items()} for p in layers]
+    nt = min(wl.T, 64)  # per step: one layer, 64 tokens through the experts
+    for i in range(a.warmup):
+        oracle_sample_rate(wl, xs, lc, budget_s=1e9, max_layers=1, n_tokens=nt, seed=i)
+    t0 = time.perf_counter()
+    rates = []
+    sample = ""
+    for i in range(a.steps):
+        r, sample, _ = oracle_sample_rate(wl, xs, lc, budget_s=1e9, max_layers=1, n_tokens=nt,
+                                          seed=1000 + i)
+        rates.append(r)
+    el = time.perf_counter() - t0
+    value = statistics.mean(rates)
+    cores = blas_threads()
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": el * 1e3 / a.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k,
+                   "d_ff": wl.d_ff, "layers": wl.layers, "gate_mode": wl.gate_mode},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": "per step: " + sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    a = parse_args()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)
+
+
+if __name__ == "__main__":
+    main()

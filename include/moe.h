@@ -1,0 +1,196 @@
+/*
+ * moe.h - C ABI of libmoe.so: the Mixture-of-Experts layer forward on one B200 (sm_100a),
+ *         "route + pack + compute + combine".
+ *
+ * The operation ("271,104 Routes: What I Missed About Mixture-of-Experts", sections 1-3;
+ * "Mixture of Experts: Routing, Dispatch, and Load Balancing", sections 2-4):
+ *   z      = x W_r^T + bias                          router logits        [T, E]
+ *   ids, g = top-k of z, gate weights (3 modes)      routing              [T, k]
+ *   pack   = rows of x duplicated per kept route and grouped by expert   [R, d]
+ *   H      = SiLU(X_p Wg_e^T) * (X_p Wu_e^T)         per expert segment   [R, F]
+ *   Y      = H Wd_e^T                                per expert segment   [R, d]
+ *   y[t]   = sum_j g[t,j] Y[row(t,j)] (+ shared expert) (+ x[t])          [T, d]
+ *
+ * Conventions shared by every entry point
+ *   Memory      Every pointer argument is a DEVICE pointer owned by the caller unless
+ *               stated otherwise.  The library never allocates device memory.
+ *   Layout      Row-major, densely packed.  Weights use nn.Linear storage [out, in]
+ *               ("Mixture of Experts: Routing, Dispatch, and Load Balancing", section 1:
+ *               the math form W_router [d, N] is stored as [N, d]); per-expert weights
+ *               are stacked along a leading expert axis.
+ *   Types       dtype MOE_BF16: x, weights, packed rows, H, Y and y are bf16 (fp32
+ *               accumulation).  dtype MOE_F32: all of those are fp32.  Gates and the
+ *               logit bias are always fp32; ids, rows and offsets are int32.
+ *   Streams     Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *               default stream).  Host-side validation errors are returned at once and
+ *               nothing is launched.  Errors found on the device (bad expert id, a
+ *               bounded wait that ran out) are recorded in the status word at the start
+ *               of the workspace; read it with moe_get_device_status.
+ *   Workspace   `ws` is caller-owned device memory of at least moe_workspace_bytes(cfg)
+ *               bytes, 256-byte aligned.  Its first 256 bytes must be zero before first
+ *               use (moe_workspace_init does this).  Calls that share a workspace must be
+ *               ordered on one stream.
+ *   Determinism The same inputs give bit-identical outputs (no floating-point atomics;
+ *               packed positions come from an ordered count, not from atomic arrival).
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Compatible with cudaStream_t without including CUDA headers. */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID = 1,        /* null pointer, non-positive size, k > E, bad enum       */
+  MOE_ERR_UNSUPPORTED = 2,    /* valid but outside what the kernels handle (see below)   */
+  MOE_ERR_WORKSPACE = 3,      /* workspace null or misaligned                             */
+  MOE_ERR_CUDA = 4,           /* a CUDA runtime/driver call or a launch failed            */
+  MOE_ERR_BAD_EXPERT_ID = 5,  /* device: an id outside [0, E) or repeated within a token  */
+  MOE_ERR_TIMEOUT = 6         /* device: a bounded wait ran out; the kernel returned early */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Where the softmax sits ("MoE Inference Visualized", The Router; "Mixture of Experts:
+ * Routing, Dispatch, and Load Balancing", section 3; "Mixture-of-experts routing",
+ * The gate).  Ranking is always on the logits, ties to the lower expert index.     */
+typedef enum {
+  MOE_GATE_SOFTMAX_TOPK = 0,        /* g = softmax over all E, taken at the top-k        */
+  MOE_GATE_SOFTMAX_TOPK_RENORM = 1, /* ... divided by the sum over the top-k             */
+  MOE_GATE_TOPK_SOFTMAX = 2         /* g = softmax over the k selected logits only       */
+} moe_gate_mode;
+
+typedef struct {
+  int32_t T;            /* tokens in this call (>= 1)                                   */
+  int32_t d;            /* model width                                                   */
+  int32_t E;            /* routed experts, 1..256                                        */
+  int32_t k;            /* experts per token, 1..min(E, 32)                              */
+  int32_t d_ff;         /* expert hidden width F                                         */
+  int32_t dtype;        /* moe_dtype                                                     */
+  int32_t gate_mode;    /* moe_gate_mode                                                 */
+  int32_t capacity;     /* < 0: dropless; else C >= 0 rows per expert (see moe_capacity) */
+  int32_t has_shared;   /* 1: one always-on shared expert, gate 1, never dropped          */
+  int32_t add_residual; /* 1: y = x + MoE(x)                                              */
+} moe_config;
+/* Supported shapes (else MOE_ERR_UNSUPPORTED): bf16 needs d % 128 == 0 and
+ * d_ff % 128 == 0; fp32 needs d % 4 == 0 and d_ff % 4 == 0.                            */
+
+/* Capacity C = ceil(phi * T * k / E), phi = phi_num / phi_den, in exact integer
+ * arithmetic ("Mixture-of-experts routing", Capacity; "Mixture-of-Experts: routing and
+ * capacity", Capacity: ceil(8*2/4 * 1.25) = 5).  Returns -1 on invalid arguments.      */
+int32_t moe_capacity(int32_t T, int32_t k, int32_t E, int32_t phi_num, int32_t phi_den);
+
+/* Upper bound on packed rows R: T*k, or E*C when capacity >= 0 and that is smaller.
+ * Buffers of packed rows (x_packed, row_token) need this many rows; H and y_packed need
+ * moe_max_rows + T rows when has_shared (the shared expert's rows follow the routed). */
+int64_t moe_max_rows(const moe_config* cfg);
+
+/* Bytes of workspace that moe_forward needs (it keeps every intermediate there); the
+ * staged calls need only the leading scratch part, which this also covers.
+ * Returns 0 for an invalid config.                                                      */
+size_t moe_workspace_bytes(const moe_config* cfg);
+
+/* Zero the status word and scratch header of a workspace (async on `stream`).          */
+moe_status moe_workspace_init(void* ws, moe_stream_t stream);
+
+/* Route: z = x W_r^T + bias, top-k ids (descending logit, ties to the lower index) and
+ * gates ("271,104 Routes...", section 2 The Router; "Mixture-of-Experts: routing and
+ * capacity", Router / Top-k and mixture).
+ *   x         [T, d]  dtype          w_router [E, d] dtype      logit_bias [E] fp32 or NULL
+ *   ids       [T, k]  int32 (out)    gates    [T, k] fp32 (out), slot j = j-th largest   */
+moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router,
+                     const float* logit_bias, int32_t* ids, float* gates, void* ws,
+                     moe_stream_t stream);
+
+/* Pack: per-expert demand, arrival-order positions (token order), capacity mask and
+ * the expert-major packed copy of x ("271,104 Routes...", section 3 Dispatch, and its
+ * subsection on capacity; "Mixture-of-Experts: routing and capacity", Worked case).
+ *   ids        [T, k] int32 (in; ids outside [0,E) or repeated in a token are dropped and
+ *              flagged MOE_ERR_BAD_EXPERT_ID in the status word)
+ *   x_packed   [moe_max_rows, d] dtype (out): row offsets[e] + p holds x[t] for the p-th
+ *              kept route of expert e (tokens ascending)
+ *   row_token  [moe_max_rows] int32 (out): token of each packed row
+ *   route_row  [T, k] int32 (out): packed row of route (t, j), -1 when dropped
+ *   offsets    [E + 2] int32 (out): segment starts; offsets[E] = R (kept routes);
+ *              offsets[E+1] = R + T with a shared expert, else R
+ *   demand     [E] int32 (out): routes asking for each expert before capacity           */
+moe_status moe_dispatch(const moe_config* cfg, const void* x, const int32_t* ids,
+                        void* x_packed, int32_t* row_token, int32_t* route_row,
+                        int32_t* offsets, int32_t* demand, void* ws, moe_stream_t stream);
+
+/* Compute: the SwiGLU expert FFNs as grouped GEMMs over the ragged expert segments
+ * ("MoE Inference Visualized", Expert Execution: down(SiLU(gate(x)) * up(x));
+ * "271,104 Routes...", section 3: one dense matmul per expert batch).
+ *   x          [T, d] (A operand of the shared expert; may be NULL without one)
+ *   x_packed   [moe_max_rows, d]       offsets [E + 2] from moe_dispatch (device)
+ *   w_gate, w_up [E, F, d]   w_down [E, d, F]
+ *   shared_gate, shared_up [F, d], shared_down [d, F]: NULL unless has_shared
+ *   h          [moe_max_rows (+T), F] dtype (out, intermediate SiLU(g)*u)
+ *   y_packed   [moe_max_rows (+T), d] dtype (out); the shared expert's row for token t
+ *              is offsets[E] + t.  Rows past offsets[E+1] are not written.              */
+moe_status moe_expert_ffn(const moe_config* cfg, const void* x, const void* x_packed,
+                          const int32_t* offsets, const void* w_gate, const void* w_up,
+                          const void* w_down, const void* shared_gate, const void* shared_up,
+                          const void* shared_down, void* h, void* y_packed, void* ws,
+                          moe_stream_t stream);
+
+/* Combine: y[t] = sum_{j kept} gates[t,j] * y_packed[route_row[t,j]], summed in slot order
+ * in fp32, + y_packed[offsets[E] + t] with a shared expert, + x[t] with add_residual
+ * ("271,104 Routes...", section 1: y = sum p_i E_i(x); section 3: apply the gate weights
+ * and restore the original token order; "Mixture-of-Experts: routing and capacity",
+ * Top-k and mixture: output = weighted sum + shared + residual).
+ *   residual   [T, d] (x) or NULL unless add_residual     y [T, d] dtype (out)           */
+moe_status moe_combine(const moe_config* cfg, const void* y_packed, const int32_t* route_row,
+                       const float* gates, const int32_t* offsets, const void* residual,
+                       void* y, moe_stream_t stream);
+
+/* The whole layer in one call: route -> pack -> compute -> combine, all intermediates in
+ * `ws`, no host synchronisation.  ids_out / gates_out / demand_out / offsets_out are
+ * optional copies of the routing metadata ([T,k], [T,k], [E], [E+2]; NULL to skip).    */
+moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_router,
+                       const float* logit_bias, const void* w_gate, const void* w_up,
+                       const void* w_down, const void* shared_gate, const void* shared_up,
+                       const void* shared_down, void* y, int32_t* ids_out, float* gates_out,
+                       int32_t* demand_out, int32_t* offsets_out, void* ws,
+                       moe_stream_t stream);
+
+/* moe_forward that also records caller-created CUDA events (cudaEvent_t handles, e.g.
+ * created with timing enabled) on `stream` around its kernels, for live per-kernel timing:
+ * events[0] before the first kernel, events[i] after kernel i, i = 1..5 in the order
+ * route, pack, gate/up GEMM, down GEMM, combine.  n_events must be 6.                   */
+moe_status moe_forward_profiled(const moe_config* cfg, const void* x, const void* w_router,
+                                const float* logit_bias, const void* w_gate, const void* w_up,
+                                const void* w_down, const void* shared_gate,
+                                const void* shared_up, const void* shared_down, void* y,
+                                int32_t* ids_out, float* gates_out, int32_t* demand_out,
+                                int32_t* offsets_out, void* const* events, int32_t n_events,
+                                void* ws, moe_stream_t stream);
+
+/* Synchronise `stream`, copy the device status word of `ws` to *status_out (a moe_status)
+ * and, if clear != 0, reset it to MOE_OK.  Returns MOE_ERR_CUDA if the copy fails.      */
+moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t clear,
+                                 int32_t* status_out);
+
+/* Test hook for failure detection: launch one CTA that waits on an mbarrier nothing
+ * arrives at, bounded by `limit_ns` nanoseconds (1e3..1e10).  The wait runs out, the
+ * kernel records MOE_ERR_TIMEOUT in the status word of `ws` and returns normally, so
+ * the context stays usable.  It exercises the same bounded-wait routine the GEMM uses. */
+moe_status moe_debug_bounded_wait(void* ws, int64_t limit_ns, moe_stream_t stream);
+
+/* Static string for a status code. */
+const char* moe_status_string(moe_status s);
+
+/* Library version, for the binding's load check. */
+int32_t moe_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H_ */

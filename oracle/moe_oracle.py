@@ -344,6 +344,7 @@ def moe_stack(x0, layers: list, k: int, mode: str, C: int | None = None,
     infos = []
     for p in layers:
         y, info = moe_layer(x, p, k, mode, C, add_residual=True)
+        info["x_in"] = x
         x = round_to_bf16(y) if bf16_activations else y
         infos.append(info)
     return x, infos

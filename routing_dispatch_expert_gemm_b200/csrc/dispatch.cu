@@ -1,0 +1,209 @@
+// Pack: per-expert demand, arrival-order positions, capacity mask, expert-major offsets,
+// and the scatter of duplicated token rows into expert batches.
+//
+// Sources: "271,104 Routes: What I Missed About Mixture-of-Experts", section 3 Dispatch
+// (route table of token, expert, position, gate; group by expert; bincount + cumsum
+// segment ends) and its subsection on expert capacity; "Mixture-of-Experts: routing and
+// capacity", Capacity and Worked case (arrival order decides which route is dropped);
+// "Mixture-of-experts routing", Capacity (C = ceil(phi T k / E)).
+//
+// Positions are deterministic without ordered atomics: the position of route (t, j) in
+// expert e is the number of earlier tokens that chose e, i.e.
+//   (routes to e in earlier token tiles)  +  popcount(bitmask of earlier tokens of this
+//   tile that chose e).
+// The first term is an exclusive prefix over a per-tile histogram; every CTA computes
+// the prefix it needs directly from the histogram (bounded to 16384 entries), so no
+// separate scan launch and no inter-CTA waiting is needed.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+int tok_tile_for(int T, int E) {
+  // The per-expert token bitmasks of one tile must also fit in 48 KB of shared memory.
+  const long long max_tt = static_cast<long long>(48 * 1024 / 4 / E) * 32;
+  int tt = 16;
+  while (static_cast<long long>((T + tt - 1) / tt) * E > 16384 && 2LL * tt <= max_tt) tt *= 2;
+  return tt;
+}
+
+namespace {
+
+constexpr int kThreads = 256;
+
+// A route is valid if its expert id is in range and not repeated earlier in the token.
+__device__ __forceinline__ bool route_valid(const int32_t* ids_row, int j, int e, int E) {
+  if (e < 0 || e >= E) return false;
+  for (int q = 0; q < j; ++q)
+    if (ids_row[q] == e) return false;
+  return true;
+}
+
+__global__ void __launch_bounds__(kThreads)
+    hist_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int tok_tile,
+                int32_t* __restrict__ tile_hist, int32_t* status) {
+  __shared__ int s_hist[256];
+  const int tile = blockIdx.x;
+  const int tok0 = tile * tok_tile;
+  const int ntok = min(tok_tile, T - tok0);
+  for (int e = threadIdx.x; e < E; e += kThreads) s_hist[e] = 0;
+  __syncthreads();
+  for (int r = threadIdx.x; r < ntok * k; r += kThreads) {
+    const int t = tok0 + r / k, j = r % k;
+    const int32_t* row = ids + static_cast<size_t>(t) * k;
+    const int e = row[j];
+    if (route_valid(row, j, e, E))
+      atomicAdd(&s_hist[e], 1);
+    else
+      record_status(status, MOE_ERR_BAD_EXPERT_ID);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kThreads)
+    tile_hist[static_cast<size_t>(tile) * E + e] = s_hist[e];
+}
+
+struct ScatterArgs {
+  const void* x;
+  const int32_t* ids;
+  const int32_t* tile_hist;
+  int T, d, k, E, tok_tile, num_tiles, capacity, has_shared;
+  void* x_packed;
+  int32_t* row_token;
+  int32_t* route_row;
+  int32_t* offsets;
+  int32_t* demand;
+  int32_t* status;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
+  constexpr int VEC = Vec<T>::N;
+  __shared__ int s_pre[256];   // routes to e in earlier tiles
+  __shared__ int s_tot[256];   // routes to e in all tiles (demand)
+  __shared__ int s_off[257];   // segment starts over kept routes
+  __shared__ int s_rows[8][32];
+  extern __shared__ uint32_t s_mask[];  // [E][words]: bit = token of this tile chose e
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tile = blockIdx.x;
+  const int tok0 = tile * a.tok_tile;
+  const int ntok = min(a.tok_tile, a.T - tok0);
+  const int words = (a.tok_tile + 31) / 32;
+  const int E = a.E, k = a.k;
+
+  for (int e = tid; e < E; e += kThreads) { s_pre[e] = 0; s_tot[e] = 0; }
+  for (int w = tid; w < E * words; w += kThreads) s_mask[w] = 0;
+  __syncthreads();
+
+  // 1. prefix (tiles < this one) and total per expert, split over all threads
+  {
+    const int nparts = kThreads / E;  // >= 1 since E <= 256
+    if (tid < nparts * E) {
+      const int e = tid % E, part = tid / E;
+      int pre = 0, tot = 0;
+      for (int i = part; i < a.num_tiles; i += nparts) {
+        const int h = __ldg(a.tile_hist + static_cast<size_t>(i) * E + e);
+        tot += h;
+        pre += (i < tile) ? h : 0;
+      }
+      atomicAdd(&s_pre[e], pre);
+      atomicAdd(&s_tot[e], tot);
+    }
+  }
+  // 2. bitmask of this tile's tokens per expert
+  for (int r = tid; r < ntok * k; r += kThreads) {
+    const int tl = r / k, j = r % k;
+    const int32_t* row = a.ids + static_cast<size_t>(tok0 + tl) * k;
+    const int e = row[j];
+    if (route_valid(row, j, e, E)) atomicOr(&s_mask[e * words + (tl >> 5)], 1u << (tl & 31));
+  }
+  __syncthreads();
+
+  // 3. kept counts -> exclusive scan -> offsets (warp 0, 32 experts per step)
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      int kept = 0;
+      if (e < E) kept = (a.capacity < 0) ? s_tot[e] : min(s_tot[e], a.capacity);
+      int incl = kept;
+#pragma unroll
+      for (int s = 1; s < 32; s <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, s);
+        if (lane >= s) incl += o;
+      }
+      if (e < E) s_off[e] = carry + incl - kept;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_off[E] = carry;
+  }
+  __syncthreads();
+  if (tile == 0) {
+    for (int e = tid; e <= E; e += kThreads) a.offsets[e] = s_off[e];
+    if (tid == 0) a.offsets[E + 1] = s_off[E] + (a.has_shared ? a.T : 0);
+    for (int e = tid; e < E; e += kThreads) a.demand[e] = s_tot[e];
+  }
+
+  // 4. per token (one warp): rows of its k routes, then copy x[t] to each kept row
+  const T* __restrict__ X = static_cast<const T*>(a.x);
+  T* __restrict__ XP = static_cast<T*>(a.x_packed);
+  const int nvec = a.d / VEC;
+  for (int tl = warp; tl < ntok; tl += 8) {
+    const int t = tok0 + tl;
+    if (lane < k) {
+      const int32_t* row = a.ids + static_cast<size_t>(t) * k;
+      const int e = row[lane];
+      int r = -1;
+      if (route_valid(row, lane, e, E)) {
+        const uint32_t* m = s_mask + e * words;
+        int rank = __popc(m[tl >> 5] & ((1u << (tl & 31)) - 1u));
+        for (int w = 0; w < (tl >> 5); ++w) rank += __popc(m[w]);
+        const int pos = s_pre[e] + rank;
+        if (a.capacity < 0 || pos < a.capacity) {
+          r = s_off[e] + pos;
+          a.row_token[r] = t;
+        }
+      }
+      a.route_row[static_cast<size_t>(t) * k + lane] = r;
+      s_rows[warp][lane] = r;
+    }
+    __syncwarp();
+    const T* src = X + static_cast<size_t>(t) * a.d;
+    for (int c = lane; c < nvec; c += 32) {
+      const uint4 v = ld_vec(src + c * VEC);
+      for (int j = 0; j < k; ++j) {
+        const int r = s_rows[warp][j];
+        if (r >= 0) st_vec(XP + static_cast<size_t>(r) * a.d + c * VEC, v);
+      }
+    }
+    __syncwarp();
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch_hist(const moe_config& c, const int32_t* ids, int32_t* tile_hist,
+                                 int32_t* status, cudaStream_t s) {
+  const int tt = tok_tile_for(c.T, c.E);
+  const int grid = (c.T + tt - 1) / tt;
+  hist_kernel<<<grid, kThreads, 0, s>>>(ids, c.T, c.k, c.E, tt, tile_hist, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_scatter(const moe_config& c, const void* x, const int32_t* ids,
+                                    const int32_t* tile_hist, void* x_packed,
+                                    int32_t* row_token, int32_t* route_row, int32_t* offsets,
+                                    int32_t* demand, int32_t* status, cudaStream_t s) {
+  const int tt = tok_tile_for(c.T, c.E);
+  const int grid = (c.T + tt - 1) / tt;
+  ScatterArgs a{x, ids, tile_hist, c.T, c.d, c.k, c.E, tt, grid, c.capacity, c.has_shared,
+                x_packed, row_token, route_row, offsets, demand, status};
+  const size_t smem = static_cast<size_t>(c.E) * ((tt + 31) / 32) * sizeof(uint32_t);
+  if (c.dtype == MOE_BF16)
+    scatter_kernel<__nv_bfloat16><<<grid, kThreads, smem, s>>>(a);
+  else
+    scatter_kernel<float><<<grid, kThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

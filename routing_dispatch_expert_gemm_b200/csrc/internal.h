@@ -1,0 +1,65 @@
+// Host-side declarations shared by the libmoe translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+// Token tile of the router / dispatch kernels: 16 * 2^j tokens, the smallest such that
+// the per-tile expert histogram (num_tiles x E int32) stays within 16384 entries.  Every
+// dispatch CTA reads the whole histogram to form its own prefix, so this bounds that work.
+int tok_tile_for(int T, int E);
+inline int num_tiles_for(int T, int E) {
+  const int tt = tok_tile_for(T, E);
+  return (T + tt - 1) / tt;
+}
+
+cudaError_t launch_router(const moe_config& c, const void* x, const void* w_router,
+                          const float* bias, int32_t* ids, float* gates, int32_t* tile_hist,
+                          int32_t* status, cudaStream_t s);
+
+cudaError_t launch_dispatch_hist(const moe_config& c, const int32_t* ids, int32_t* tile_hist,
+                                 int32_t* status, cudaStream_t s);
+
+cudaError_t launch_dispatch_scatter(const moe_config& c, const void* x, const int32_t* ids,
+                                    const int32_t* tile_hist, void* x_packed,
+                                    int32_t* row_token, int32_t* route_row, int32_t* offsets,
+                                    int32_t* demand, int32_t* status, cudaStream_t s);
+
+cudaError_t launch_combine(const moe_config& c, const void* y_packed, const int32_t* route_row,
+                           const float* gates, const int32_t* offsets, const void* residual,
+                           void* y, cudaStream_t s);
+
+struct FfnArgs {
+  const void* x;          // [T, d] (shared expert's A operand)
+  const void* x_packed;   // [Rmax, d]
+  const int32_t* offsets; // [E + 2]
+  const void* w_gate;     // [E, F, d]
+  const void* w_up;       // [E, F, d]
+  const void* w_down;     // [E, d, F]
+  const void* s_gate;     // [F, d] or null
+  const void* s_up;       // [F, d] or null
+  const void* s_down;     // [d, F] or null
+  void* h;                // [Rmax (+T), F]
+  void* y_packed;         // [Rmax (+T), d]
+  int64_t rmax;           // rows of x_packed
+  int32_t* status;
+};
+
+// fp32 path: CUDA-core grouped GEMMs.  `mid` (may be null) is recorded between the
+// gate/up and the down GEMM.
+cudaError_t launch_ffn_simt(const moe_config& c, const FfnArgs& a, cudaStream_t s,
+                            cudaEvent_t mid = nullptr);
+// bf16 path: persistent tcgen05/TMEM grouped GEMMs fed by TMA.
+cudaError_t launch_ffn_sm100(const moe_config& c, const FfnArgs& a, cudaStream_t s,
+                             cudaEvent_t mid = nullptr);
+
+cudaError_t launch_debug_wait(int32_t* status, int64_t limit_ns, cudaStream_t s);
+
+// Default bound on every in-kernel wait (nanoseconds).
+constexpr int64_t kWaitLimitNs = 2000000000LL;
+
+}  // namespace moe

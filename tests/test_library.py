@@ -1,0 +1,106 @@
+"""CPU checks of the C-ABI library: it builds, loads, exports every symbol that
+include/moe.h declares, and its host-side logic (validation, capacity, sizes) is right.
+No call here launches work on a GPU: every call either is pure host arithmetic or fails
+validation before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from oracle import moe_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def native():
+    from routing_dispatch_expert_gemm_b200 import build, native
+    build.build()
+    native.lib()
+    return native
+
+
+def header_functions():
+    with open(os.path.join(ROOT, "include", "moe.h")) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(native):
+    declared = header_functions()
+    assert len(declared) >= 12
+    assert sorted(native.EXPORTS) == declared
+    lib = ctypes.CDLL(native.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert native.moe_abi_version() == 1
+
+
+def test_library_is_sm100a_build(native):
+    from routing_dispatch_expert_gemm_b200 import build
+    assert "arch=compute_100a,code=sm_100a" in build.ARCH
+
+
+def test_capacity_matches_oracle(native):
+    for T in (1, 7, 8, 16, 256, 1412, 4096, 8192):
+        for k in (1, 2, 8):
+            for E in (1, 4, 8, 32, 64):
+                for num, den in ((1, 2), (1, 1), (5, 4), (3, 2), (2, 1)):
+                    assert native.moe_capacity(T, k, E, num, den) == O.capacity(T, k, E, num, den)
+    assert native.moe_capacity(8, 2, 4, 5, 4) == 5
+    assert native.moe_capacity(8, 2, 0, 1, 1) == -1
+    assert native.moe_capacity(8, 2, 4, 1, 0) == -1
+
+
+def test_validation_and_sizes(native):
+    cfg = native.make_config(64, 64, 4, 2, 128, dtype="f32", gate_mode="softmax_topk_renorm")
+    assert native.moe_max_rows(cfg) == 128
+    ws = native.moe_workspace_bytes(cfg)
+    assert ws > 256 and ws % 256 == 0
+    capped = native.make_config(4096, 768, 4, 1, 2432, capacity=512, gate_mode="softmax_topk")
+    assert native.moe_max_rows(capped) == 2048
+    zero = native.make_config(16, 128, 4, 1, 128, capacity=0)
+    assert native.moe_max_rows(zero) == 1
+    shared = native.make_config(16, 4096, 64, 2, 32768, has_shared=True,
+                                gate_mode="softmax_topk_renorm")
+    assert native.moe_workspace_bytes(shared) > native.moe_workspace_bytes(
+        native.make_config(16, 4096, 64, 2, 32768, gate_mode="softmax_topk_renorm"))
+    bad = [native.make_config(0, 64, 4, 2, 128),                  # T < 1
+           native.make_config(8, 64, 4, 5, 128),                  # k > E
+           native.make_config(8, 64, 4, 2, 128, gate_mode="topk_softmax")]
+    bad[2].gate_mode = 7
+    for c in bad:
+        assert native.moe_workspace_bytes(c) == 0
+    unsupported = [native.make_config(8, 96, 4, 2, 128),          # bf16 needs d % 128
+                   native.make_config(8, 128, 300, 2, 128),       # E > 256
+                   native.make_config(8, 64, 4, 2, 130, dtype="f32")]
+    for c in unsupported:
+        assert native.moe_workspace_bytes(c) == 0
+
+
+def test_errors_return_before_any_launch(native):
+    lib = native.lib()
+    cfg = native.make_config(8, 128, 4, 2, 128)
+    fake = 1 << 20  # never dereferenced: validation fails first
+    # k > E: invalid config
+    badk = native.make_config(8, 128, 4, 5, 128)
+    assert lib.moe_route(ctypes.byref(badk), fake, fake, None, fake, fake, 256 * 4096, None) == 1
+    # unaligned / missing workspace
+    assert lib.moe_route(ctypes.byref(cfg), fake, fake, None, fake, fake, 12345, None) == 3
+    assert lib.moe_route(ctypes.byref(cfg), fake, fake, None, fake, fake, None, None) == 3
+    # null required pointers
+    assert lib.moe_route(ctypes.byref(cfg), None, fake, None, fake, fake, 4096, None) == 1
+    assert lib.moe_dispatch(ctypes.byref(cfg), fake, None, fake, fake, fake, fake, fake,
+                            4096, None) == 1
+    assert lib.moe_combine(ctypes.byref(cfg), fake, fake, fake, None, None, None, None) == 1
+    res = native.make_config(8, 128, 4, 2, 128, add_residual=True)
+    assert lib.moe_combine(ctypes.byref(res), fake, fake, fake, fake, None, fake, None) == 1
+    sh = native.make_config(8, 128, 4, 2, 128, has_shared=True)
+    assert lib.moe_expert_ffn(ctypes.byref(sh), fake, fake, fake, fake, fake, fake, None, None,
+                              None, fake, fake, 4096, None) == 1
+    assert lib.moe_forward(ctypes.byref(cfg), fake, fake, None, fake, fake, fake, None, None,
+                           None, None, None, None, None, None, 4096, None) == 1
+    assert lib.moe_debug_bounded_wait(4096, 10, None) == 1
+    assert native.moe_status_string(6).startswith("a bounded")
