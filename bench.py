@@ -50,7 +50,8 @@ def parse_args():
     ap.add_argument("--profiled-steps", type=int, default=20,
                     help="timed steps that also record per-kernel events")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--graph", action="store_true", help="replay the step as a CUDA graph")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="launch through the library call by call instead of replaying a CUDA graph")
     a = ap.parse_args()
     a.warmup = max(a.warmup, 3)
     return a
@@ -261,6 +262,7 @@ def run_ours(a):
     stream = torch.cuda.current_stream(dev)
 
     def step(xin, evs=None):
+        st_ = torch.cuda.current_stream(dev)
         h = xin
         for l, p in enumerate(layers):
             y = ybuf[l % 2]
@@ -268,9 +270,9 @@ def run_ours(a):
                     p["shared_gate"], p["shared_up"], p["shared_down"], y, None, None,
                     demand[l], offsets[l])
             if evs is None:
-                N.moe_forward(*args, ws, stream)
+                N.moe_forward(*args, ws, st_)
             else:
-                N.moe_forward_profiled(*args, evs[l], ws, stream)
+                N.moe_forward_profiled(*args, evs[l], ws, st_)
             h = y
         return h
 
@@ -289,12 +291,39 @@ def run_ours(a):
         raise RuntimeError(f"device status {st} after warm-up")
 
     nprof = min(a.profiled_steps, a.steps)
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(L)]
-           for _ in range(nprof)]
-    for s in evs:  # create the handles before timing
-        for l in s:
-            for e in l:
-                e.record(stream)
+    evs = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
+            for _ in range(L)] for _ in range(nprof)]
+    for s_ in evs:  # create the handles before capture / timing
+        for l_ in s_:
+            for e_ in l_:
+                e_.record(stream)
+    torch.cuda.synchronize(dev)
+
+    # The step as CUDA graphs: one plain graph, plus one graph per profiled step (each
+    # with its own events).  Replaying removes the host launch overhead of 5 x layers
+    # library calls per step; every kernel still launches on every replay.
+    graphs = []
+    g_plain = None
+    if a.graph:
+        cs = torch.cuda.Stream(dev)
+        g_plain = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_plain, stream=cs):
+            step(x)
+        for i in range(nprof):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cs):
+                step(x, evs[i])
+            graphs.append(g)
+        for _ in range(2):
+            g_plain.replay()
+        torch.cuda.synchronize(dev)
+
+    def run_step(i):
+        if a.graph:
+            (graphs[i] if i < nprof else g_plain).replay()
+        else:
+            step(x, evs[i] if i < nprof else None)
+
     step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(a.steps)]
     bus = None
@@ -310,12 +339,12 @@ def run_ours(a):
         dist.barrier()
     torch.cuda.synchronize(dev)
     t0 = time.time()
-    for s in range(a.steps):
+    for s_i in range(a.steps):
         if flush is not None:
             flush.zero_()
-        step_ev[s][0].record(stream)
-        step(x, evs[s] if s < nprof else None)
-        step_ev[s][1].record(stream)
+        step_ev[s_i][0].record(stream)
+        run_step(s_i)
+        step_ev[s_i][1].record(stream)
     torch.cuda.synchronize(dev)
     t1 = time.time()
     if world > 1:
@@ -380,17 +409,31 @@ def run_ours(a):
     x_host = x.cpu().pin_memory()
     y_host = torch.empty_like(x_host).pin_memory()
     x_dev = torch.empty_like(x)
-    for _ in range(2):
+    g_e2e = None
+    if a.graph:
+        g_e2e = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_e2e, stream=cs):
+            out_e2e = step(x_dev)
+    else:
+        out_e2e = None
+
+    def e2e_step():
         x_dev.copy_(x_host, non_blocking=True)
-        y_host.copy_(step(x_dev), non_blocking=True)
+        if g_e2e is not None:
+            g_e2e.replay()
+            y_host.copy_(out_e2e, non_blocking=True)
+        else:
+            y_host.copy_(step(x_dev), non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(a.steps):
-        x_dev.copy_(x_host, non_blocking=True)
-        y_host.copy_(step(x_dev), non_blocking=True)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
@@ -400,6 +443,8 @@ def run_ours(a):
     nbytes = x.numel() * x.element_size()
     e2e = {"value": world * wl.T * L / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
            "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes}
+    ok_out = torch.isfinite(y_host.float()).all().item()
+    del graphs, g_plain, g_e2e
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
@@ -422,11 +467,12 @@ def run_ours(a):
                    "d_ff": wl.d_ff, "layers": L, "gate_mode": wl.gate_mode,
                    "capacity": cap, "shared_expert": wl.has_shared,
                    "residual": wl.add_residual, "parallelism": f"replicas{world}",
+                   "cuda_graph": a.graph,
                    "l2": ("flushed between steps" if flush is not None else
                           f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB of weights per step)")},
         "roofline": roofline, "kernels": breakdown, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": a.steps * L * 5, "clocks": clk,
-        "routes_per_step": int(dem.sum()),
+        "routes_per_step": int(dem.sum()), "output_finite": bool(ok_out),
     }
     print(json.dumps(out), flush=True)
 

@@ -65,6 +65,19 @@ __device__ __forceinline__ void st_vec(void* p, const uint4& v) {
 }
 
 // ---------------------------------------------------------------------------------
+// cp.async (16-byte global -> shared copies that bypass registers)
+// ---------------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------------
 // Time and shared-memory addresses
 // ---------------------------------------------------------------------------------
 __device__ __forceinline__ uint64_t global_timer_ns() {

@@ -22,7 +22,7 @@ namespace moe {
 int tok_tile_for(int T, int E) {
   // The per-expert token bitmasks of one tile must also fit in 48 KB of shared memory.
   const long long max_tt = static_cast<long long>(48 * 1024 / 4 / E) * 32;
-  int tt = 16;
+  int tt = 8;
   while (static_cast<long long>((T + tt - 1) / tt) * E > 16384 && 2LL * tt <= max_tt) tt *= 2;
   return tt;
 }
@@ -78,10 +78,12 @@ struct ScatterArgs {
 template <typename T>
 __global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
   constexpr int VEC = Vec<T>::N;
+  constexpr int kSub = 32;     // tokens whose rows are resolved per copy round
+  constexpr int kBatch = 8;    // histogram loads in flight per thread
   __shared__ int s_pre[256];   // routes to e in earlier tiles
   __shared__ int s_tot[256];   // routes to e in all tiles (demand)
   __shared__ int s_off[257];   // segment starts over kept routes
-  __shared__ int s_rows[8][32];
+  __shared__ int s_rows[kSub][32];
   extern __shared__ uint32_t s_mask[];  // [E][words]: bit = token of this tile chose e
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -95,16 +97,25 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
   for (int w = tid; w < E * words; w += kThreads) s_mask[w] = 0;
   __syncthreads();
 
-  // 1. prefix (tiles < this one) and total per expert, split over all threads
+  // 1. prefix (tiles < this one) and total per expert, split over all threads with
+  //    kBatch independent loads in flight per thread
   {
     const int nparts = kThreads / E;  // >= 1 since E <= 256
     if (tid < nparts * E) {
       const int e = tid % E, part = tid / E;
       int pre = 0, tot = 0;
-      for (int i = part; i < a.num_tiles; i += nparts) {
-        const int h = __ldg(a.tile_hist + static_cast<size_t>(i) * E + e);
-        tot += h;
-        pre += (i < tile) ? h : 0;
+      for (int i0 = part; i0 < a.num_tiles; i0 += nparts * kBatch) {
+        int h[kBatch];
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+          const int i = i0 + q * nparts;
+          h[q] = (i < a.num_tiles) ? __ldg(a.tile_hist + static_cast<size_t>(i) * E + e) : 0;
+        }
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+          tot += h[q];
+          pre += (i0 + q * nparts < tile) ? h[q] : 0;
+        }
       }
       atomicAdd(&s_pre[e], pre);
       atomicAdd(&s_tot[e], tot);
@@ -144,39 +155,42 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
     for (int e = tid; e < E; e += kThreads) a.demand[e] = s_tot[e];
   }
 
-  // 4. per token (one warp): rows of its k routes, then copy x[t] to each kept row
+  // 4. rows of kSub tokens' routes, then the copy of those tokens: one thread per
+  //    (token, 16-byte vector), one load and up to k stores
   const T* __restrict__ X = static_cast<const T*>(a.x);
   T* __restrict__ XP = static_cast<T*>(a.x_packed);
   const int nvec = a.d / VEC;
-  for (int tl = warp; tl < ntok; tl += 8) {
-    const int t = tok0 + tl;
-    if (lane < k) {
+  for (int s0 = 0; s0 < ntok; s0 += kSub) {
+    const int nsub = min(kSub, ntok - s0);
+    for (int r = tid; r < nsub * k; r += kThreads) {
+      const int ts = r / k, j = r - ts * k;
+      const int tl = s0 + ts, t = tok0 + tl;
       const int32_t* row = a.ids + static_cast<size_t>(t) * k;
-      const int e = row[lane];
-      int r = -1;
-      if (route_valid(row, lane, e, E)) {
+      const int e = row[j];
+      int out = -1;
+      if (route_valid(row, j, e, E)) {
         const uint32_t* m = s_mask + e * words;
         int rank = __popc(m[tl >> 5] & ((1u << (tl & 31)) - 1u));
         for (int w = 0; w < (tl >> 5); ++w) rank += __popc(m[w]);
         const int pos = s_pre[e] + rank;
         if (a.capacity < 0 || pos < a.capacity) {
-          r = s_off[e] + pos;
-          a.row_token[r] = t;
+          out = s_off[e] + pos;
+          a.row_token[out] = t;
         }
       }
-      a.route_row[static_cast<size_t>(t) * k + lane] = r;
-      s_rows[warp][lane] = r;
+      a.route_row[static_cast<size_t>(t) * k + j] = out;
+      s_rows[ts][j] = out;
     }
-    __syncwarp();
-    const T* src = X + static_cast<size_t>(t) * a.d;
-    for (int c = lane; c < nvec; c += 32) {
-      const uint4 v = ld_vec(src + c * VEC);
+    __syncthreads();
+    for (int idx = tid; idx < nsub * nvec; idx += kThreads) {
+      const int ts = idx / nvec, c = idx - ts * nvec;
+      const uint4 v = ld_vec(X + static_cast<size_t>(tok0 + s0 + ts) * a.d + c * VEC);
       for (int j = 0; j < k; ++j) {
-        const int r = s_rows[warp][j];
+        const int r = s_rows[ts][j];
         if (r >= 0) st_vec(XP + static_cast<size_t>(r) * a.d + c * VEC, v);
       }
     }
-    __syncwarp();
+    __syncthreads();
   }
 }
 

@@ -391,7 +391,8 @@ cudaError_t launch_ffn_sm100(const moe_config& c, const FfnArgs& f, cudaStream_t
             f.status, kWaitLimitNs};
   cudaError_t e = launch_gemm<0, 256>(m1, p1, mt_bound * (c.d_ff / 128), s);
   if (e != cudaSuccess) return e;
-  if (mid != nullptr && (e = cudaEventRecord(mid, s)) != cudaSuccess) return e;
+  if (mid != nullptr && (e = cudaEventRecordWithFlags(mid, s, cudaEventRecordExternal)) != cudaSuccess)
+    return e;
 
   // down:  A = H [rows_h, F]
   Maps m2;

@@ -8,7 +8,7 @@
 
 namespace moe {
 
-// Token tile of the router / dispatch kernels: 16 * 2^j tokens, the smallest such that
+// Token tile of the router / dispatch kernels: 8 * 2^j tokens, the smallest such that
 // the per-tile expert histogram (num_tiles x E int32) stays within 16384 entries.  Every
 // dispatch CTA reads the whole histogram to form its own prefix, so this bounds that work.
 int tok_tile_for(int T, int E);

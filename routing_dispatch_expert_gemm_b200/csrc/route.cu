@@ -6,8 +6,8 @@
 // (softmax, topk, normalised weighted sum); "MoE Inference Visualized", The Router;
 // "Mixture-of-experts routing", The gate.
 //
-// Design: one warp per token (two tokens per warp per pass).  A block of EP experts'
-// router rows is staged in shared memory in d-chunks and shared by the CTA's 16 tokens;
+// Design: one warp per token (8 tokens per CTA round).  A block of EP experts' router
+// rows is staged in shared memory (cp.async) in d-chunks and shared by the CTA's tokens;
 // each lane accumulates fp32 partial dot products for all EP experts over its slice of d
 // (16-byte loads of x), then a reduce-scatter across the warp leaves the logit of expert
 // (lane mod EP) on each lane.  Top-k is k rounds of a warp arg-max ordered by (logit
@@ -21,8 +21,9 @@ namespace moe {
 namespace {
 
 constexpr int kThreads = 256;       // 8 warps
-constexpr int kTokPerWarp = 2;      // tokens per warp per sub-batch
+constexpr int kTokPerWarp = 1;      // tokens per warp per sub-batch
 constexpr int kSubTokens = 8 * kTokPerWarp;
+constexpr int kXBatch = 4;          // x vectors loaded together per lane
 constexpr int kWChunkBytes = 64 * 1024;
 
 struct RouterArgs {
@@ -107,25 +108,39 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(RouterArgs a) {
         for (int v = tid; v < EP * ncv; v += kThreads) {
           const int e = v / ncv, c = v - e * ncv;
           const int ge = p * EP + e;
-          s_w[e * dcv + c] = (ge < a.E) ? ld_vec(W + static_cast<size_t>(ge) * a.d + d0 + c * VEC)
-                                        : make_uint4(0, 0, 0, 0);
+          if (ge < a.E)
+            cp_async_16(&s_w[e * dcv + c], W + static_cast<size_t>(ge) * a.d + d0 + c * VEC);
+          else
+            s_w[e * dcv + c] = make_uint4(0, 0, 0, 0);
         }
+        cp_async_wait_all();
         __syncthreads();
 #pragma unroll
         for (int i = 0; i < kTokPerWarp; ++i) {
           if (tok[i] >= tok_end) continue;
           const Tin* xr = X + static_cast<size_t>(tok[i]) * a.d + d0;
-          for (int c = lane; c < ncv; c += 32) {
-            float xf[VEC];
-            Vec<Tin>::to_f32(ld_vec(xr + c * VEC), xf);
+          for (int c0 = lane; c0 < ncv; c0 += 32 * kXBatch) {
+            uint4 xv[kXBatch];
 #pragma unroll
-            for (int e = 0; e < EP; ++e) {
-              float wf[VEC];
-              Vec<Tin>::to_f32(s_w[e * dcv + c], wf);
-              float s = acc[i][e];
+            for (int u = 0; u < kXBatch; ++u) {
+              const int c = c0 + 32 * u;
+              xv[u] = (c < ncv) ? ld_vec(xr + c * VEC) : make_uint4(0, 0, 0, 0);
+            }
 #pragma unroll
-              for (int q = 0; q < VEC; ++q) s = fmaf(xf[q], wf[q], s);
-              acc[i][e] = s;
+            for (int u = 0; u < kXBatch; ++u) {
+              const int c = c0 + 32 * u;
+              if (c >= ncv) break;
+              float xf[VEC];
+              Vec<Tin>::to_f32(xv[u], xf);
+#pragma unroll
+              for (int e = 0; e < EP; ++e) {
+                float wf[VEC];
+                Vec<Tin>::to_f32(s_w[e * dcv + c], wf);
+                float s = acc[i][e];
+#pragma unroll
+                for (int q = 0; q < VEC; ++q) s = fmaf(xf[q], wf[q], s);
+                acc[i][e] = s;
+              }
             }
           }
         }
