@@ -96,12 +96,9 @@ moe_status ffn(const moe_config& c, const FfnArgs& f, cudaStream_t s, cudaEvent_
                                          : launch_ffn_simt(c, f, s, mid));
 }
 
-// External records: inside stream capture they become event-record nodes of the graph, so
-// the events still time the kernels when the forward is replayed as a CUDA graph.
 moe_status record(void* const* events, int i, cudaStream_t s) {
   if (events == nullptr) return MOE_OK;
-  return cuda_status(
-      cudaEventRecordWithFlags(static_cast<cudaEvent_t>(events[i]), s, cudaEventRecordExternal));
+  return cuda_status(record_event(static_cast<cudaEvent_t>(events[i]), s));
 }
 
 moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_router,

@@ -65,6 +65,18 @@ __device__ __forceinline__ void st_vec(void* p, const uint4& v) {
 }
 
 // ---------------------------------------------------------------------------------
+// Event records that also time correctly inside CUDA-graph stream capture: while the
+// stream is capturing they become external event-record nodes of the graph.
+// ---------------------------------------------------------------------------------
+inline cudaError_t record_event(cudaEvent_t ev, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(s, &cs);
+  if (e != cudaSuccess) return e;
+  return cudaEventRecordWithFlags(
+      ev, s, cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault);
+}
+
+// ---------------------------------------------------------------------------------
 // cp.async (16-byte global -> shared copies that bypass registers)
 // ---------------------------------------------------------------------------------
 __device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gmem_src) {

@@ -116,8 +116,7 @@ cudaError_t launch_ffn_simt(const moe_config& c, const FfnArgs& f, cudaStream_t 
   simt_kernel<0><<<grid1, kThreads, 0, s>>>(g);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (mid != nullptr && (e = cudaEventRecordWithFlags(mid, s, cudaEventRecordExternal)) != cudaSuccess)
-    return e;
+  if (mid != nullptr && (e = record_event(mid, s)) != cudaSuccess) return e;
   SimtArgs g2{static_cast<const float*>(f.h), static_cast<const float*>(f.h), f.offsets,
               static_cast<const float*>(f.w_down), nullptr, static_cast<const float*>(f.s_down),
               nullptr, static_cast<float*>(f.y_packed), c.E, nseg, c.d_ff, c.d};

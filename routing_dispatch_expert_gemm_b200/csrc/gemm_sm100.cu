@@ -6,15 +6,16 @@
 // "271,104 Routes: What I Missed About Mixture-of-Experts", section 3 (one dense matmul per
 // expert batch) and section 5 (once expert batches are large the matmuls dominate).
 //
-// Kernel shape (one CTA per SM, persistent, 6 warps):
-//   warp 4    TMA producer: A tile [128 rows x 64 K] and B tile [BN rows x 64 K] per
+// Kernel shape (one CTA per SM, persistent, 10 warps):
+//   warp 8    TMA producer: A tile [128 rows x 64 K] and B tile [BN rows x 64 K] per
 //             stage, 128-byte swizzle, into a STAGES-deep shared-memory ring.
-//   warp 5    MMA issuer: tcgen05.mma kind::f16 (bf16 in, fp32 accumulate) M=128,
+//   warp 9    MMA issuer: tcgen05.mma kind::f16 (bf16 in, fp32 accumulate) M=128,
 //             N=BN, K=16 x 4 per stage into a tensor-memory accumulator; two accumulators
 //             (2 x BN columns) so the epilogue of one tile overlaps the MMAs of the next.
-//   warps 0-3 epilogue: tcgen05.ld of the accumulator (warp w owns TMEM lanes 32w..32w+31,
-//             i.e. tile rows), SiLU(gate)*up or plain conversion, bf16 stores of the
-//             rows that belong to the segment.
+//   warps 0-7 epilogue: tcgen05.ld of the accumulator (warp w owns TMEM lanes
+//             32(w%4)..+31, i.e. tile rows, and half the columns), SiLU(gate)*up or plain
+//             conversion to bf16, staged through shared memory so that the stores to
+//             global memory are 64-byte row segments, only for rows of the segment.
 // In the gate/up GEMM the B tile stacks 128 rows of W_gate over the same 128 rows of
 // W_up, so one N=256 MMA produces both halves side by side in TMEM and the SwiGLU is
 // applied in the epilogue with no extra pass.
@@ -34,7 +35,12 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = one 128-byte swizzle row
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;                    // two per TMEM lane quarter
+constexpr int kProducerWarp = kEpiWarps;        // warp 8
+constexpr int kMmaWarp = kEpiWarps + 1;         // warp 9
+constexpr int kThreads = 32 * (kEpiWarps + 2);
+constexpr int kStageRowBytes = 80;              // 64 B of a row chunk + 16 B pad (no bank conflicts)
+constexpr int kEpiStageBytes = 32 * kStageRowBytes;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int kBoxRows = 128;
 constexpr int kMaxSeg = 260;
@@ -64,7 +70,8 @@ struct Cfg {
   static constexpr int STAGES = (BN == 256) ? 4 : 6;
   static constexpr int OUT_COLS = (MODE == 0) ? BN / 2 : BN;
   static constexpr int TMEM_COLS = 2 * BN;
-  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 256 + 2 * kMaxSeg * 4;
+  static constexpr int SMEM =
+      1024 + STAGES * STAGE_BYTES + kEpiWarps * kEpiStageBytes + 256 + 2 * kMaxSeg * 4;
 };
 
 __device__ __forceinline__ int find_seg(const int* pre, int nseg, int tile) {
@@ -76,7 +83,10 @@ __device__ __forceinline__ int find_seg(const int* pre, int nseg, int tile) {
   return lo;
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.f + __expf(-g)); }
+// SiLU(g) = g / (1 + e^-g) with the fast approximate exponential and division (about 2 ulp
+// in fp32; the result is rounded to bf16).  For g -> -inf the denominator overflows and the
+// quotient is 0, the limit of SiLU.
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.f + __expf(-g)); }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -92,7 +102,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = base;
   uint8_t* sB = base + C::STAGES * A_BYTES;
-  uint8_t* ctl = sB + C::STAGES * C::B_BYTES;
+  uint8_t* sEpi = sB + C::STAGES * C::B_BYTES;  // per epilogue warp: 32 rows x 80 B
+  uint8_t* ctl = sEpi + kEpiWarps * kEpiStageBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(ctl);
   uint64_t* empty = full + 8;
   uint64_t* tfull = empty + 8;
@@ -109,17 +120,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 4); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], kEpiWarps); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     tma_prefetch_desc(&maps.a_routed);
     tma_prefetch_desc(&maps.b0_routed);
     if (MODE == 0) tma_prefetch_desc(&maps.b1_routed);
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -148,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int total = s_pre[p.nseg];
 
-  if (warp == 4 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     // ------------------------------------------------------------ TMA producer
     int stage = 0;
     uint32_t phase = 0;
@@ -192,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_bounded(&full[s], par, nullptr, p.limit_ns, p.status);
       }
     }
-  } else if (warp == 5 && lane == 0) {
+  } else if (warp == kMmaWarp && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
     int stage = 0, acc = 0;
@@ -227,11 +238,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(drain);
       mbar_wait_bounded(drain, 0, nullptr, p.limit_ns, p.status);
     }
-  } else if (warp < 4) {
+  } else if (warp < kEpiWarps) {
     // ------------------------------------------------------------ epilogue
+    // Warp w reads TMEM lanes 32*(w%4).. (tile rows) and half of the output columns
+    // (w/4).  Each 32 x 32 chunk is converted in registers, staged in this warp's padded
+    // shared-memory slice and written back as 64-byte row segments (4 lanes per row).
+    const int quarter = warp & 3, half = warp >> 2;
+    constexpr int COLS = C::OUT_COLS / 2;  // output columns of this warp
+    uint8_t* stage_mem = sEpi + warp * kEpiStageBytes;
     int acc = 0;
     uint32_t acc_phase = 0;
-    const int r_in_tile = warp * 32 + lane;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       const int s = find_seg(s_pre, p.nseg, tile);
       const int rows = s_row0[s + 1] - s_row0[s];
@@ -243,49 +259,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) +
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-      const bool store = r_in_tile < rows - m * BM;
-      __nv_bfloat16* orow = p.out + static_cast<size_t>(s_row0[s] + m * BM + r_in_tile) * p.ldo +
-                            static_cast<size_t>(n) * C::OUT_COLS;
-      if (MODE == 0) {
+      const int valid = rows - m * BM - quarter * 32;  // rows of this warp's 32 that exist
+      __nv_bfloat16* out0 = p.out + static_cast<size_t>(s_row0[s] + m * BM + quarter * 32) * p.ldo +
+                            static_cast<size_t>(n) * C::OUT_COLS + half * COLS;
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN / 2; c0 += 32) {
+      for (int c0 = 0; c0 < COLS; c0 += 32) {
+        uint32_t o[16];
+        if (MODE == 0) {
           uint32_t g[32], u[32];
-          tmem_ld_32x32b_x32(t_row + c0, g);
-          tmem_ld_32x32b_x32(t_row + BN / 2 + c0, u);
+          tmem_ld_32x32b_x32(t_row + half * COLS + c0, g);
+          tmem_ld_32x32b_x32(t_row + BN / 2 + half * COLS + c0, u);
           tmem_ld_wait();
-          uint32_t o[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float h0 = silu_f(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
             const float h1 = silu_f(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
             o[i] = pack_bf16(h0, h1);
           }
-          if (store) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-          }
-        }
-      } else {
-#pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 32) {
+        } else {
           uint32_t v[32];
-          tmem_ld_32x32b_x32(t_row + c0, v);
+          tmem_ld_32x32b_x32(t_row + half * COLS + c0, v);
           tmem_ld_wait();
-          uint32_t o[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             o[i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-          if (store) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-          }
         }
+        // stage: lane = row, 64 bytes
+        uint4* srow = reinterpret_cast<uint4*>(stage_mem + lane * kStageRowBytes);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) srow[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+        __syncwarp();
+        // write back: 4 lanes per row, 8 rows per instruction, 64 contiguous bytes per row
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = i * 8 + (lane >> 2), q = lane & 3;
+          const uint4 v = *reinterpret_cast<const uint4*>(stage_mem + r * kStageRowBytes + q * 16);
+          if (r < valid)
+            *reinterpret_cast<uint4*>(out0 + static_cast<size_t>(r) * p.ldo + c0 + q * 8) = v;
+        }
+        __syncwarp();
       }
       tc_fence_before();
       __syncwarp();
@@ -297,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem_base, C::TMEM_COLS);
+  if (warp == kMmaWarp) tmem_dealloc(tmem_base, C::TMEM_COLS);
 }
 
 __global__ void debug_wait_kernel(int32_t* status, int64_t limit_ns) {
@@ -391,8 +405,7 @@ cudaError_t launch_ffn_sm100(const moe_config& c, const FfnArgs& f, cudaStream_t
             f.status, kWaitLimitNs};
   cudaError_t e = launch_gemm<0, 256>(m1, p1, mt_bound * (c.d_ff / 128), s);
   if (e != cudaSuccess) return e;
-  if (mid != nullptr && (e = cudaEventRecordWithFlags(mid, s, cudaEventRecordExternal)) != cudaSuccess)
-    return e;
+  if (mid != nullptr && (e = record_event(mid, s)) != cudaSuccess) return e;
 
   // down:  A = H [rows_h, F]
   Maps m2;

@@ -23,7 +23,9 @@ namespace {
 constexpr int kThreads = 256;       // 8 warps
 constexpr int kTokPerWarp = 1;      // tokens per warp per sub-batch
 constexpr int kSubTokens = 8 * kTokPerWarp;
-constexpr int kXBatch = 4;          // x vectors loaded together per lane
+// x vectors loaded together per lane: fewer for 32 experts per pass so that two CTAs
+// (16 warps) fit on an SM without spilling the 32 partial sums.
+template <int EP> constexpr int kXBatch = (EP >= 32) ? 2 : 4;
 constexpr int kWChunkBytes = 64 * 1024;
 
 struct RouterArgs {
@@ -119,15 +121,15 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(RouterArgs a) {
         for (int i = 0; i < kTokPerWarp; ++i) {
           if (tok[i] >= tok_end) continue;
           const Tin* xr = X + static_cast<size_t>(tok[i]) * a.d + d0;
-          for (int c0 = lane; c0 < ncv; c0 += 32 * kXBatch) {
-            uint4 xv[kXBatch];
+          for (int c0 = lane; c0 < ncv; c0 += 32 * kXBatch<EP>) {
+            uint4 xv[kXBatch<EP>];
 #pragma unroll
-            for (int u = 0; u < kXBatch; ++u) {
+            for (int u = 0; u < kXBatch<EP>; ++u) {
               const int c = c0 + 32 * u;
               xv[u] = (c < ncv) ? ld_vec(xr + c * VEC) : make_uint4(0, 0, 0, 0);
             }
 #pragma unroll
-            for (int u = 0; u < kXBatch; ++u) {
+            for (int u = 0; u < kXBatch<EP>; ++u) {
               const int c = c0 + 32 * u;
               if (c >= ncv) break;
               float xf[VEC];

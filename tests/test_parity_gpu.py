@@ -324,3 +324,32 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     x, (p,) = I.make_inputs(W["tiny_fp32"], seed=0, device="cuda", layers=1)
     out = forward_gpu(cfg, x, p, ws)
     assert out["status"] == 0
+
+
+def test_forward_profiled_matches_forward_and_times_kernels():
+    """moe_forward_profiled gives the same bits as moe_forward, called directly and when
+    captured into a CUDA graph, and its events time every kernel."""
+    wl = W["granite24"].with_(layers=1)
+    x, (p,) = I.make_inputs(wl, seed=4, device="cuda", layers=1)
+    cfg = config_for(wl)
+    ref = forward_gpu(cfg, x, p)
+    ws = N.workspace(cfg)
+    args = lambda y: (cfg, x, p["w_router"], p["logit_bias"], p["w_gate"], p["w_up"], p["w_down"],
+                      p["shared_gate"], p["shared_up"], p["shared_down"], y, None, None, None, None)
+    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
+    y1 = torch.empty_like(x)
+    N.moe_forward_profiled(*args(y1), evs, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, ref["y"])
+    times = [evs[i].elapsed_time(evs[i + 1]) for i in range(5)]
+    assert all(t > 0 for t in times), times
+    y2 = torch.empty_like(x)
+    g = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream()
+    with torch.cuda.graph(g, stream=cs):
+        N.moe_forward_profiled(*args(y2), evs, ws)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y2, ref["y"])
+    assert all(evs[i].elapsed_time(evs[i + 1]) > 0 for i in range(5))
+    assert N.moe_get_device_status(ws) == 0
