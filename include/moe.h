@@ -184,6 +184,31 @@ moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t clear,
  * the context stays usable.  It exercises the same bounded-wait routine the GEMM uses. */
 moe_status moe_debug_bounded_wait(void* ws, int64_t limit_ns, moe_stream_t stream);
 
+/* moe_dispatch without a workspace, for callers that cannot allocate device memory:
+ * plugins that receive only their input and output buffers from a framework that owns
+ * all device memory, runtimes with a memory budget fixed before start-up, or hot paths
+ * that must not call an allocator (allocation may synchronise or take a global lock).
+ * The pages have no counterpart; it is the pack step of moe_dispatch with the same
+ * arguments and outputs, minus `ws`.
+ *   Scratch: the per-token-tile expert histogram lives in a fixed 64 KiB array inside the
+ *   library (16384 int32 entries, held by every device that loads the library until the
+ *   process exits).  Configurations whose histogram, ceil(T / tile) * E entries with the
+ *   token tile of moe_dispatch, exceeds 16384 entries are rejected with
+ *   MOE_ERR_UNSUPPORTED; nothing is launched then.
+ *   Set-up: the first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any stream capture.
+ *   Sharing: every call on a device uses the same array and it keeps the last call's
+ *   contents; nothing in it needs to start at zero because each call rewrites the entries
+ *   it reads.  Calls that overlap on the GPU (other streams, other host threads) race on
+ *   the array: order them on one stream.
+ *   status: device int32 or NULL.  If given, it must hold 0 before the call; a bad expert
+ *   id is recorded there as MOE_ERR_BAD_EXPERT_ID (the route is dropped).
+ * Calls no cudaMalloc, cudaFree or other allocating routine.                            */
+moe_status moe_dispatch_noalloc(const moe_config* cfg, const void* x, const int32_t* ids,
+                                void* x_packed, int32_t* row_token, int32_t* route_row,
+                                int32_t* offsets, int32_t* demand, int32_t* status,
+                                moe_stream_t stream);
+
 /* Static string for a status code. */
 const char* moe_status_string(moe_status s);
 

@@ -22,8 +22,8 @@ GATE_MODES = {"softmax_topk": 0, "softmax_topk_renorm": 1, "topk_softmax": 2}
 # Every symbol include/moe.h declares (checked by the CPU test suite).
 EXPORTS = ("moe_capacity", "moe_max_rows", "moe_workspace_bytes", "moe_workspace_init",
            "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_forward",
-           "moe_forward_profiled", "moe_get_device_status", "moe_debug_bounded_wait", "moe_status_string",
-           "moe_abi_version")
+           "moe_forward_profiled", "moe_get_device_status", "moe_debug_bounded_wait",
+           "moe_dispatch_noalloc", "moe_status_string", "moe_abi_version")
 
 
 class MoeError(RuntimeError):
@@ -75,6 +75,7 @@ def lib() -> ctypes.CDLL:
             "moe_forward_profiled": (_I32, [_CFG] + [_P] * 14 + [ctypes.POINTER(_P), _I32, _P, _P]),
             "moe_get_device_status": (_I32, [_P, _P, _I32, ctypes.POINTER(_I32)]),
             "moe_debug_bounded_wait": (_I32, [_P, ctypes.c_int64, _P]),
+            "moe_dispatch_noalloc": (_I32, [_CFG] + [_P] * 8 + [_P]),
             "moe_status_string": (ctypes.c_char_p, [_I32]),
             "moe_abi_version": (_I32, []),
         }
@@ -193,6 +194,16 @@ def moe_get_device_status(ws, stream=None, clear=False) -> int:
 def moe_debug_bounded_wait(ws, limit_ns, stream=None):
     _check(lib().moe_debug_bounded_wait(_ptr(ws), int(limit_ns), _stream(stream)),
            "moe_debug_bounded_wait")
+
+
+def moe_dispatch_noalloc(cfg, x, ids, x_packed, row_token, route_row, offsets, demand,
+                         status=None, stream=None):
+    """moe_dispatch without a workspace: for callers that cannot allocate device memory.
+    Its scratch is a fixed array inside libmoe.so (see include/moe.h)."""
+    _check(lib().moe_dispatch_noalloc(ctypes.byref(cfg), _ptr(x), _ptr(ids), _ptr(x_packed),
+                                      _ptr(row_token), _ptr(route_row), _ptr(offsets),
+                                      _ptr(demand), _ptr(status), _stream(stream)),
+           "moe_dispatch_noalloc")
 
 
 def workspace(cfg: MoeConfig, device="cuda"):
