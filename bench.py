@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--profiled-steps", type=int, default=20,
                     help="timed steps that also record per-kernel events")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="override the workload's layer count (a stack of fewer layers)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="launch through the library call by call instead of replaying a CUDA graph")
     a = ap.parse_args()
@@ -250,6 +252,8 @@ def run_ours(a):
     N.lib()
 
     wl = I.WORKLOADS[a.workload]
+    if a.layers is not None:
+        wl = wl.with_(layers=a.layers)
     L = wl.layers
     x, layers = I.make_inputs(wl, seed=a.seed + rank, device=dev)
     cap = -1 if wl.phi is None else N.moe_capacity(wl.T, wl.k, wl.E, *wl.phi)

@@ -39,6 +39,8 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
   __shared__ float s_g[kMaxTok][32];
   const int t0 = blockIdx.x * a.tpc;
   const int ntok = min(a.tpc, a.T - t0);
+  pdl_trigger();
+  pdl_wait();
   for (int i = threadIdx.x; i < ntok * a.k; i += kThreads) {
     const int tl = i / a.k, j = i - tl * a.k;
     s_row[tl][j] = __ldg(a.route_row + static_cast<size_t>(t0) * a.k + i);
@@ -105,11 +107,15 @@ cudaError_t launch_combine(const moe_config& c, const void* y_packed, const int3
   CombineArgs a{y_packed, route_row, gates, offsets, c.add_residual ? residual : nullptr,
                 y, c.T, c.d, c.k, c.E, c.has_shared, tpc};
   const int grid = (c.T + tpc - 1) / tpc;
+  static bool configured = false;
+  if (!configured) {
+    prefer_max_shared(combine_kernel<__nv_bfloat16>);
+    prefer_max_shared(combine_kernel<float>);
+    configured = true;
+  }
   if (c.dtype == MOE_BF16)
-    combine_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(a);
-  else
-    combine_kernel<float><<<grid, kThreads, 0, s>>>(a);
-  return cudaGetLastError();
+    return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(kThreads), 0, s, a);
+  return launch_pdl(combine_kernel<float>, dim3(grid), dim3(kThreads), 0, s, a);
 }
 
 }  // namespace moe

@@ -77,6 +77,47 @@ inline cudaError_t record_event(cudaEvent_t ev, cudaStream_t s) {
 }
 
 // ---------------------------------------------------------------------------------
+// Every kernel of the library asks for the largest shared-memory carveout, so that
+// consecutive kernels (the GEMMs need ~220 KB) do not make the SMs switch L1/shared
+// configuration between launches.  Called once per kernel from its launcher.
+// ---------------------------------------------------------------------------------
+template <typename K>
+inline cudaError_t prefer_max_shared(K kernel) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              cudaSharedmemCarveoutMaxShared);
+}
+
+// ---------------------------------------------------------------------------------
+// Programmatic dependent launch.  Every kernel of the forward is launched so that it may
+// start while the previous kernel on the stream is still finishing: it runs its prologue
+// (barrier init, tensor-memory allocation, descriptor prefetch), then pdl_wait(), which
+// returns once the previous kernel has completed and its writes are visible.  No kernel
+// reads data produced by, or writes data read by, an earlier kernel before pdl_wait().
+// pdl_trigger() lets the next kernel be scheduled early.  Both are no-ops when the
+// kernel was launched without the attribute.
+// ---------------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// ---------------------------------------------------------------------------------
 // cp.async (16-byte global -> shared copies that bypass registers)
 // ---------------------------------------------------------------------------------
 __device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gmem_src) {

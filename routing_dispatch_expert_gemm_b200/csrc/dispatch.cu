@@ -11,21 +11,14 @@
 // expert e is the number of earlier tokens that chose e, i.e.
 //   (routes to e in earlier token tiles)  +  popcount(bitmask of earlier tokens of this
 //   tile that chose e).
-// The first term is an exclusive prefix over a per-tile histogram; every CTA computes
-// the prefix it needs directly from the histogram (bounded to 16384 entries), so no
-// separate scan launch and no inter-CTA waiting is needed.
+// The first term is an exclusive prefix over the per-128-token-tile histogram; every CTA
+// computes the prefix it needs directly from the histogram (ceil(T/128) x E entries), so
+// no separate scan launch and no inter-CTA waiting is needed.  Pack CTAs cover 8-token
+// sub-tiles of a histogram tile, so the copy work spreads over many SMs.
 #include "common.cuh"
 #include "internal.h"
 
 namespace moe {
-
-int tok_tile_for(int T, int E) {
-  // The per-expert token bitmasks of one tile must also fit in 48 KB of shared memory.
-  const long long max_tt = static_cast<long long>(48 * 1024 / 4 / E) * 32;
-  int tt = 8;
-  while (static_cast<long long>((T + tt - 1) / tt) * E > 16384 && 2LL * tt <= max_tt) tt *= 2;
-  return tt;
-}
 
 namespace {
 
@@ -47,6 +40,8 @@ __global__ void __launch_bounds__(kThreads)
   const int tok0 = tile * tok_tile;
   const int ntok = min(tok_tile, T - tok0);
   for (int e = threadIdx.x; e < E; e += kThreads) s_hist[e] = 0;
+  pdl_trigger();
+  pdl_wait();
   __syncthreads();
   for (int r = threadIdx.x; r < ntok * k; r += kThreads) {
     const int t = tok0 + r / k, j = r % k;
@@ -75,26 +70,31 @@ struct ScatterArgs {
   int32_t* status;
 };
 
+constexpr int kSubTok = 8;  // tokens packed per CTA
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
   constexpr int VEC = Vec<T>::N;
-  constexpr int kSub = 32;     // tokens whose rows are resolved per copy round
   constexpr int kBatch = 8;    // histogram loads in flight per thread
+  constexpr int kWords = kHistTile / 32;
   __shared__ int s_pre[256];   // routes to e in earlier tiles
   __shared__ int s_tot[256];   // routes to e in all tiles (demand)
   __shared__ int s_off[257];   // segment starts over kept routes
-  __shared__ int s_rows[kSub][32];
-  extern __shared__ uint32_t s_mask[];  // [E][words]: bit = token of this tile chose e
+  __shared__ int s_rows[kSubTok][32];
+  __shared__ uint32_t s_mask[256 * kWords];  // [E][words]: bit = token of the tile chose e
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tile = blockIdx.x;
-  const int tok0 = tile * a.tok_tile;
-  const int ntok = min(a.tok_tile, a.T - tok0);
-  const int words = (a.tok_tile + 31) / 32;
+  const int t_begin = blockIdx.x * kSubTok;
+  const int nsub = min(kSubTok, a.T - t_begin);
+  const int tile = t_begin / kHistTile;
+  const int tile0 = tile * kHistTile;
+  const int ntile = min(kHistTile, a.T - tile0);
   const int E = a.E, k = a.k;
 
   for (int e = tid; e < E; e += kThreads) { s_pre[e] = 0; s_tot[e] = 0; }
-  for (int w = tid; w < E * words; w += kThreads) s_mask[w] = 0;
+  for (int w = tid; w < E * kWords; w += kThreads) s_mask[w] = 0;
+  pdl_trigger();
+  pdl_wait();
   __syncthreads();
 
   // 1. prefix (tiles < this one) and total per expert, split over all threads with
@@ -121,12 +121,12 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
       atomicAdd(&s_tot[e], tot);
     }
   }
-  // 2. bitmask of this tile's tokens per expert
-  for (int r = tid; r < ntok * k; r += kThreads) {
+  // 2. bitmask of the histogram tile's tokens per expert
+  for (int r = tid; r < ntile * k; r += kThreads) {
     const int tl = r / k, j = r % k;
-    const int32_t* row = a.ids + static_cast<size_t>(tok0 + tl) * k;
+    const int32_t* row = a.ids + static_cast<size_t>(tile0 + tl) * k;
     const int e = row[j];
-    if (route_valid(row, j, e, E)) atomicOr(&s_mask[e * words + (tl >> 5)], 1u << (tl & 31));
+    if (route_valid(row, j, e, E)) atomicOr(&s_mask[e * kWords + (tl >> 5)], 1u << (tl & 31));
   }
   __syncthreads();
 
@@ -149,48 +149,61 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
     if (lane == 0) s_off[E] = carry;
   }
   __syncthreads();
-  if (tile == 0) {
+  if (blockIdx.x == 0) {
     for (int e = tid; e <= E; e += kThreads) a.offsets[e] = s_off[e];
     if (tid == 0) a.offsets[E + 1] = s_off[E] + (a.has_shared ? a.T : 0);
     for (int e = tid; e < E; e += kThreads) a.demand[e] = s_tot[e];
   }
 
-  // 4. rows of kSub tokens' routes, then the copy of those tokens: one thread per
-  //    (token, 16-byte vector), one load and up to k stores
+  // 4. rows of this CTA's tokens' routes
+  for (int r = tid; r < nsub * k; r += kThreads) {
+    const int ts = r / k, j = r - ts * k;
+    const int t = t_begin + ts, tl = t - tile0;
+    const int32_t* row = a.ids + static_cast<size_t>(t) * k;
+    const int e = row[j];
+    int out = -1;
+    if (route_valid(row, j, e, E)) {
+      const uint32_t* m = s_mask + e * kWords;
+      int rank = __popc(m[tl >> 5] & ((1u << (tl & 31)) - 1u));
+      for (int w = 0; w < (tl >> 5); ++w) rank += __popc(m[w]);
+      const int pos = s_pre[e] + rank;
+      if (a.capacity < 0 || pos < a.capacity) {
+        out = s_off[e] + pos;
+        a.row_token[out] = t;
+      }
+    }
+    a.route_row[static_cast<size_t>(t) * k + j] = out;
+    s_rows[ts][j] = out;
+  }
+  __syncthreads();
+
+  // 5. copy: one thread per (token, 16-byte vector), one load and up to k stores; loads of
+  //    kBatch vectors are issued together
   const T* __restrict__ X = static_cast<const T*>(a.x);
   T* __restrict__ XP = static_cast<T*>(a.x_packed);
   const int nvec = a.d / VEC;
-  for (int s0 = 0; s0 < ntok; s0 += kSub) {
-    const int nsub = min(kSub, ntok - s0);
-    for (int r = tid; r < nsub * k; r += kThreads) {
-      const int ts = r / k, j = r - ts * k;
-      const int tl = s0 + ts, t = tok0 + tl;
-      const int32_t* row = a.ids + static_cast<size_t>(t) * k;
-      const int e = row[j];
-      int out = -1;
-      if (route_valid(row, j, e, E)) {
-        const uint32_t* m = s_mask + e * words;
-        int rank = __popc(m[tl >> 5] & ((1u << (tl & 31)) - 1u));
-        for (int w = 0; w < (tl >> 5); ++w) rank += __popc(m[w]);
-        const int pos = s_pre[e] + rank;
-        if (a.capacity < 0 || pos < a.capacity) {
-          out = s_off[e] + pos;
-          a.row_token[out] = t;
+  const int total = nsub * nvec;
+  for (int i0 = tid; i0 < total; i0 += kThreads * kBatch) {
+    uint4 v[kBatch];
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+      const int idx = i0 + q * kThreads;
+      if (idx < total) {
+        const int ts = idx / nvec, c = idx - ts * nvec;
+        v[q] = ld_vec(X + static_cast<size_t>(t_begin + ts) * a.d + c * VEC);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+      const int idx = i0 + q * kThreads;
+      if (idx < total) {
+        const int ts = idx / nvec, c = idx - ts * nvec;
+        for (int j = 0; j < k; ++j) {
+          const int r = s_rows[ts][j];
+          if (r >= 0) st_vec(XP + static_cast<size_t>(r) * a.d + c * VEC, v[q]);
         }
       }
-      a.route_row[static_cast<size_t>(t) * k + j] = out;
-      s_rows[ts][j] = out;
     }
-    __syncthreads();
-    for (int idx = tid; idx < nsub * nvec; idx += kThreads) {
-      const int ts = idx / nvec, c = idx - ts * nvec;
-      const uint4 v = ld_vec(X + static_cast<size_t>(tok0 + s0 + ts) * a.d + c * VEC);
-      for (int j = 0; j < k; ++j) {
-        const int r = s_rows[ts][j];
-        if (r >= 0) st_vec(XP + static_cast<size_t>(r) * a.d + c * VEC, v);
-      }
-    }
-    __syncthreads();
   }
 }
 
@@ -200,24 +213,32 @@ cudaError_t launch_dispatch_hist(const moe_config& c, const int32_t* ids, int32_
                                  int32_t* status, cudaStream_t s) {
   const int tt = tok_tile_for(c.T, c.E);
   const int grid = (c.T + tt - 1) / tt;
-  hist_kernel<<<grid, kThreads, 0, s>>>(ids, c.T, c.k, c.E, tt, tile_hist, status);
-  return cudaGetLastError();
+  static bool configured = false;
+  if (!configured) {
+    prefer_max_shared(hist_kernel);
+    configured = true;
+  }
+  return launch_pdl(hist_kernel, dim3(grid), dim3(kThreads), 0, s, ids, c.T, c.k, c.E, tt,
+                    tile_hist, status);
 }
 
 cudaError_t launch_dispatch_scatter(const moe_config& c, const void* x, const int32_t* ids,
                                     const int32_t* tile_hist, void* x_packed,
                                     int32_t* row_token, int32_t* route_row, int32_t* offsets,
                                     int32_t* demand, int32_t* status, cudaStream_t s) {
-  const int tt = tok_tile_for(c.T, c.E);
-  const int grid = (c.T + tt - 1) / tt;
-  ScatterArgs a{x, ids, tile_hist, c.T, c.d, c.k, c.E, tt, grid, c.capacity, c.has_shared,
-                x_packed, row_token, route_row, offsets, demand, status};
-  const size_t smem = static_cast<size_t>(c.E) * ((tt + 31) / 32) * sizeof(uint32_t);
+  const int grid = (c.T + kSubTok - 1) / kSubTok;
+  ScatterArgs a{x, ids, tile_hist, c.T, c.d, c.k, c.E, kHistTile, num_tiles_for(c.T, c.E),
+                c.capacity, c.has_shared, x_packed, row_token, route_row, offsets, demand,
+                status};
+  static bool configured = false;
+  if (!configured) {
+    prefer_max_shared(scatter_kernel<__nv_bfloat16>);
+    prefer_max_shared(scatter_kernel<float>);
+    configured = true;
+  }
   if (c.dtype == MOE_BF16)
-    scatter_kernel<__nv_bfloat16><<<grid, kThreads, smem, s>>>(a);
-  else
-    scatter_kernel<float><<<grid, kThreads, smem, s>>>(a);
-  return cudaGetLastError();
+    return launch_pdl(scatter_kernel<__nv_bfloat16>, dim3(grid), dim3(kThreads), 0, s, a);
+  return launch_pdl(scatter_kernel<float>, dim3(grid), dim3(kThreads), 0, s, a);
 }
 
 }  // namespace moe

@@ -48,6 +48,8 @@ __global__ void __launch_bounds__(kThreads) simt_kernel(SimtArgs a) {
   __shared__ float sB0[BK][BN + 1];
   __shared__ float sB1[MODE == 0 ? BK : 1][BN + 1];
   __shared__ int s_seg, s_m;
+  pdl_trigger();
+  pdl_wait();
   if (threadIdx.x == 0) s_seg = find_segment(a.offsets, a.nseg, blockIdx.x, &s_m);
   __syncthreads();
   const int seg = s_seg;
@@ -113,16 +115,14 @@ cudaError_t launch_ffn_simt(const moe_config& c, const FfnArgs& f, cudaStream_t 
              static_cast<const float*>(f.s_gate), static_cast<const float*>(f.s_up),
              static_cast<float*>(f.h), c.E, nseg, c.d, c.d_ff};
   dim3 grid1(mtiles, (c.d_ff + BN - 1) / BN);
-  simt_kernel<0><<<grid1, kThreads, 0, s>>>(g);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(simt_kernel<0>, grid1, dim3(kThreads), 0, s, g);
   if (e != cudaSuccess) return e;
   if (mid != nullptr && (e = record_event(mid, s)) != cudaSuccess) return e;
   SimtArgs g2{static_cast<const float*>(f.h), static_cast<const float*>(f.h), f.offsets,
               static_cast<const float*>(f.w_down), nullptr, static_cast<const float*>(f.s_down),
               nullptr, static_cast<float*>(f.y_packed), c.E, nseg, c.d_ff, c.d};
   dim3 grid2(mtiles, (c.d + BN - 1) / BN);
-  simt_kernel<1><<<grid2, kThreads, 0, s>>>(g2);
-  return cudaGetLastError();
+  return launch_pdl(simt_kernel<1>, grid2, dim3(kThreads), 0, s, g2);
 }
 
 }  // namespace moe

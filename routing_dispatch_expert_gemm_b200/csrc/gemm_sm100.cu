@@ -31,6 +31,30 @@
 #include "internal.h"
 
 namespace moe {
+
+// Tensor map of a row-major bf16 matrix [rows, cols] read in boxes of 64 columns x
+// box_rows rows with 128-byte swizzle; rows outside the matrix read as zero.
+bool encode_2d_box(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows,
+                   uint32_t box_rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  if (fn == nullptr || ptr == nullptr || rows == 0 || box_rows == 0 || box_rows > 256) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 namespace {
 
 constexpr int BM = 128;
@@ -134,6 +158,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
+  pdl_trigger();
+  pdl_wait();  // offsets, A rows and the output buffer belong to earlier kernels
   if (warp == 0) {  // segment table: row starts and exclusive prefix of tile counts
     for (int i = lane; i <= p.nseg; i += 32) s_row0[i] = __ldg(p.offsets + i);
     __syncwarp();
@@ -329,31 +355,10 @@ __global__ void debug_wait_kernel(int32_t* status, int64_t limit_ns) {
 
 // ---------------------------------------------------------------- host side
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return nullptr;
-    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }();
-  return fn;
-}
-
 // Row-major bf16 matrix [rows, cols] read in boxes of 64 columns x 128 rows, 128-byte
 // swizzle; rows outside the matrix read as zero.
 bool encode_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows) {
-  auto fn = encode_fn();
-  if (fn == nullptr || ptr == nullptr || rows == 0) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {BK, kBoxRows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return encode_2d_box(m, ptr, cols, rows, kBoxRows);
 }
 
 int sm_count() {
@@ -374,12 +379,12 @@ cudaError_t launch_gemm(const Maps& maps, const Params& p, long long tiles_bound
     cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, BN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
+    prefer_max_shared(grouped_gemm_kernel<MODE, BN>);
     configured = true;
   }
   const int grid = static_cast<int>(tiles_bound < sm_count() ? (tiles_bound > 0 ? tiles_bound : 1)
                                                              : sm_count());
-  grouped_gemm_kernel<MODE, BN><<<grid, kThreads, C::SMEM, s>>>(maps, p);
-  return cudaGetLastError();
+  return launch_pdl(grouped_gemm_kernel<MODE, BN>, dim3(grid), dim3(kThreads), C::SMEM, s, maps, p);
 }
 
 }  // namespace

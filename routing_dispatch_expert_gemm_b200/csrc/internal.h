@@ -8,18 +8,20 @@
 
 namespace moe {
 
-// Token tile of the router / dispatch kernels: 8 * 2^j tokens, the smallest such that
-// the per-tile expert histogram (num_tiles x E int32) stays within 16384 entries.  Every
-// dispatch CTA reads the whole histogram to form its own prefix, so this bounds that work.
-int tok_tile_for(int T, int E);
-inline int num_tiles_for(int T, int E) {
-  const int tt = tok_tile_for(T, E);
-  return (T + tt - 1) / tt;
-}
+// Token tile of the expert histogram that connects routing and packing: 128 tokens, the
+// router's CTA tile (one TMEM lane per token).  The histogram is num_tiles x E int32.
+constexpr int kHistTile = 128;
+inline int tok_tile_for(int /*T*/, int /*E*/) { return kHistTile; }
+inline int num_tiles_for(int T, int /*E*/) { return (T + kHistTile - 1) / kHistTile; }
 
 cudaError_t launch_router(const moe_config& c, const void* x, const void* w_router,
                           const float* bias, int32_t* ids, float* gates, int32_t* tile_hist,
                           int32_t* status, cudaStream_t s);
+
+// bf16 router on tensor cores (route_sm100.cu); the fp32 router runs on CUDA cores.
+cudaError_t launch_router_sm100(const moe_config& c, const void* x, const void* w_router,
+                                const float* bias, int32_t* ids, float* gates,
+                                int32_t* tile_hist, int32_t* status, cudaStream_t s);
 
 cudaError_t launch_dispatch_hist(const moe_config& c, const int32_t* ids, int32_t* tile_hist,
                                  int32_t* status, cudaStream_t s);

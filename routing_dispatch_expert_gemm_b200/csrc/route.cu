@@ -1,5 +1,6 @@
-// Router: logits z = x W_r^T + bias, softmax and warp-level top-k with lowest-index ties,
-// gate weights in one of three modes, and a per-token-tile expert histogram for dispatch.
+// Router on CUDA cores (fp32 layers; bf16 layers use route_sm100.cu): logits
+// z = x W_r^T + bias, softmax and warp-level top-k with lowest-index ties, gate weights in
+// one of three modes, and the per-token-tile expert histogram for dispatch.
 //
 // Sources: "271,104 Routes: What I Missed About Mixture-of-Experts", section 2 The Router;
 // "Mixture of Experts: Routing, Dispatch, and Load Balancing", section 1 and section 3
@@ -85,6 +86,8 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(RouterArgs a) {
   const Tin* __restrict__ W = static_cast<const Tin*>(a.w);
 
   for (int e = tid; e < a.E; e += kThreads) s_hist[e] = 0;
+  pdl_trigger();
+  pdl_wait();
 
   for (int sub = tok0; sub < tok_end; sub += kSubTokens) {
     int tok[kTokPerWarp];
@@ -224,8 +227,7 @@ cudaError_t launch_ep(const RouterArgs& a, int grid, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  router_kernel<Tin, EP><<<grid, kThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(router_kernel<Tin, EP>, dim3(grid), dim3(kThreads), smem, s, a);
 }
 
 template <typename Tin>
@@ -252,10 +254,12 @@ cudaError_t launch_typed(RouterArgs a, cudaStream_t s) {
 
 cudaError_t launch_router(const moe_config& c, const void* x, const void* w_router,
                           const float* bias, int32_t* ids, float* gates, int32_t* tile_hist,
-                          int32_t* /*status*/, cudaStream_t s) {
-  RouterArgs a{x, w_router, bias, c.T, c.d, c.E, c.k, c.gate_mode, tok_tile_for(c.T, c.E), 0,
+                          int32_t* status, cudaStream_t s) {
+  if (c.dtype == MOE_BF16)
+    return launch_router_sm100(c, x, w_router, bias, ids, gates, tile_hist, status, s);
+  RouterArgs a{x, w_router, bias, c.T, c.d, c.E, c.k, c.gate_mode, kHistTile, 0,
                ids, gates, tile_hist};
-  return c.dtype == MOE_BF16 ? launch_typed<__nv_bfloat16>(a, s) : launch_typed<float>(a, s);
+  return launch_typed<float>(a, s);
 }
 
 }  // namespace moe

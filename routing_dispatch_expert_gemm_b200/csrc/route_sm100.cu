@@ -1,0 +1,371 @@
+// Router for bf16 layers on the 5th-generation tensor cores: logits z = x W_r^T + bias,
+// top-k (largest first, ties to the lower expert index), gates in one of three modes, and
+// the expert histogram of the 128-token tile, in one kernel.
+//
+// Sources: "271,104 Routes: What I Missed About Mixture-of-Experts", section 2 The Router
+// (a projection, topk, softmax of the selected logits); "Mixture of Experts: Routing,
+// Dispatch, and Load Balancing", section 1 (linear projection + softmax, weight stored
+// [N, d]) and section 3 (topk of the probabilities, division by the selected total);
+// "MoE Inference Visualized", The Router (the top-1 weight is the softmax probability);
+// "Mixture-of-experts routing", The gate (softmax over only the top-k).
+//
+// One CTA per 128 tokens.  The logit contraction [128 x d] x [d x E] runs as tcgen05.mma
+// with M = 128 tokens and N = E rounded up to 16 experts, fp32 accumulation in tensor
+// memory; x streams through a deep TMA ring (the router-weight tile per stage is small, so
+// up to 12 stages fit).  The epilogue gives each thread one token (one TMEM lane): it reads
+// the token's E logits in 16-column chunks, keeps a sorted top-KMAX list in registers
+// (insertion in expert order, so an equal logit never displaces an earlier expert), then
+// forms the gates and adds the token's experts to the tile histogram.  For E <= 64 the
+// token's logits stay in registers and top-k is a tournament (see topk_tournament).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+bool encode_2d_box(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows,
+                   uint32_t box_rows);
+
+namespace {
+
+constexpr int kTokens = 128;           // tokens per CTA = MMA M = TMEM lanes
+constexpr int BK = 64;                 // 128-byte swizzle rows of bf16
+constexpr int kThreads = 192;          // warps 0-3 epilogue, 4 TMA producer, 5 MMA
+#ifndef MOE_ROUTER_MAX_STAGES
+#define MOE_ROUTER_MAX_STAGES 12
+#endif
+constexpr int kMaxStages = MOE_ROUTER_MAX_STAGES;
+constexpr int A_BYTES = kTokens * BK * 2;
+constexpr int kRingBudget = 192 * 1024;
+
+struct RouteMaps {
+  CUtensorMap x;  // [T, d] bf16, box 64 x 128
+  CUtensorMap w;  // [E, d] bf16, box 64 x EN (rows >= E read as zero)
+};
+
+struct RouteParams {
+  const float* bias;
+  int T, d, E, k, EN, gate_mode, stages, tmem_cols;
+  int32_t* ids;
+  float* gates;
+  int32_t* tile_hist;
+  int32_t* status;
+  int64_t limit_ns;
+};
+
+__device__ __forceinline__ float rank_key(float z) { return isnan(z) ? -INFINITY : z; }
+
+// (v, e) ranks before (v2, e2): larger logit first, then lower expert index.
+__device__ __forceinline__ bool ranks_before(float v, int e, float v2, int e2) {
+  return v > v2 || (v == v2 && e < e2);
+}
+
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Top-k of one token's logits z[0..NV) held in registers: k rounds of a tournament
+// (binary-tree arg-max).  At every node the left child covers lower expert indices, so
+// taking the left child on equality breaks ties towards the lower index exactly; taken
+// experts are masked out.  Each round has depth log2(NV) and NV-1 independent-per-level
+// comparisons, which keeps the per-thread dependency chains short.
+template <int NV, int KMAX>
+__device__ __forceinline__ void topk_tournament(const float (&z)[NV], int E, int k, float (&tv)[KMAX],
+                                                int (&te)[KMAX]) {
+  uint64_t taken = 0;
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    if (j >= k) break;
+    float bv[NV];
+    int bi[NV];
+    bool ok[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      bv[i] = z[i];
+      bi[i] = i;
+      ok[i] = (i < E) && !((taken >> i) & 1u);
+    }
+#pragma unroll
+    for (int w = NV / 2; w >= 1; w /= 2) {
+#pragma unroll
+      for (int i = 0; i < w; ++i) {
+        const bool left = ok[2 * i] && (!ok[2 * i + 1] || bv[2 * i] >= bv[2 * i + 1]);
+        bv[i] = left ? bv[2 * i] : bv[2 * i + 1];
+        bi[i] = left ? bi[2 * i] : bi[2 * i + 1];
+        ok[i] = ok[2 * i] || ok[2 * i + 1];
+      }
+    }
+    tv[j] = bv[0];
+    te[j] = bi[0];
+    taken |= 1ull << bi[0];
+  }
+}
+
+// EN_T: compile-time logit count for E <= 64 (16, 32 or 64, whole token in registers);
+// 0 selects the general path (any E <= 256) that streams 16-logit chunks through an
+// insertion into a sorted top-KMAX list.
+template <int EN_T, int KMAX>
+__global__ void __launch_bounds__(kThreads, 1)
+    router_tc_kernel(const __grid_constant__ RouteMaps maps, const RouteParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int b_bytes = p.EN * BK * 2;
+  const int stage_bytes = A_BYTES + b_bytes;  // multiple of 1024 (EN multiple of 8)
+  uint8_t* ctl = base + p.stages * stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ctl);
+  uint64_t* empty = full + kMaxStages;
+  uint64_t* tfull = empty + kMaxStages;
+  uint64_t* drain = tfull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 8 * (2 * kMaxStages + 2));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* s_bias = reinterpret_cast<float*>(ctl + 256);
+  int* s_hist = reinterpret_cast<int*>(ctl + 256 + 256 * 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x;
+  const int k_blocks = p.d / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    mbar_init(tfull, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&maps.x);
+    tma_prefetch_desc(&maps.w);
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, p.tmem_cols);
+    tmem_relinquish();
+  }
+  pdl_trigger();
+  pdl_wait();  // x comes from the previous layer; ids/gates/hist are read by earlier kernels
+  for (int e = threadIdx.x; e < 256; e += kThreads) {
+    s_bias[e] = (e < p.E && p.bias != nullptr) ? __ldg(p.bias + e) : 0.f;
+    s_hist[e] = 0;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 4 && lane == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    bool wrapped = false, ok = true;
+    for (int kb = 0; kb < k_blocks; ++kb) {
+      if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.limit_ns, p.status)) {
+        ok = false;
+        break;
+      }
+      mbar_arrive_expect_tx(&full[stage], stage_bytes);
+      uint8_t* dst = base + stage * stage_bytes;
+      tma_load_2d(dst, &maps.x, &full[stage], kb * BK, tile * kTokens);
+      tma_load_2d(dst + A_BYTES, &maps.w, &full[stage], kb * BK, 0);
+      if (++stage == p.stages) { stage = 0; phase ^= 1u; wrapped = true; }
+    }
+    if (!ok) {
+      for (int s = 0; s < p.stages; ++s) {
+        if (!wrapped && s >= stage) continue;
+        mbar_wait_bounded(&full[s], (s < stage) ? phase : (phase ^ 1u), nullptr, p.limit_ns, p.status);
+      }
+    }
+  } else if (warp == 5 && lane == 0) {
+    // ---------------------------------------------------------------- MMA issuer
+    const uint32_t idesc = idesc_bf16_f32(kTokens, p.EN);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int kb = 0; kb < k_blocks; ++kb) {
+      if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.limit_ns, p.status)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint8_t* src = base + stage * stage_bytes;
+      const uint64_t ad = smem_desc_k_sw128(src);
+      const uint64_t bd = smem_desc_k_sw128(src + A_BYTES);
+#pragma unroll
+      for (int kk = 0; kk < BK / 16; ++kk)
+        tc_mma_bf16(tmem_base, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+      tc_commit(&empty[stage]);
+      if (++stage == p.stages) { stage = 0; phase ^= 1u; }
+    }
+    if (ok) {
+      tc_commit(tfull);
+    } else {
+      tc_commit(drain);
+      mbar_wait_bounded(drain, 0, nullptr, p.limit_ns, p.status);
+    }
+  } else if (warp < 4) {
+    // ---------------------------------------------------------------- epilogue
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait_bounded(tfull, 0, abort_flag, p.limit_ns, p.status);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok) {
+      tc_fence_after();
+      const uint32_t trow = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+      const int t = tile * kTokens + warp * 32 + lane;
+      float tv[KMAX];
+      int te[KMAX];
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) { tv[j] = -INFINITY; te[j] = 0x7fffffff; }
+      float zr[EN_T > 0 ? EN_T : 1];
+      if constexpr (EN_T > 0) {
+#pragma unroll
+        for (int c0 = 0; c0 < EN_T; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld_32x32b_x16(trow + c0, r);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) zr[c0 + j] = __uint_as_float(r[j]);
+        }
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < EN_T; ++e) zr[e] = (e < p.E) ? rank_key(zr[e] + s_bias[e]) : -INFINITY;
+        topk_tournament<EN_T, KMAX>(zr, p.E, p.k, tv, te);
+      } else {
+        for (int c0 = 0; c0 < p.EN; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld_32x32b_x16(trow + c0, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int e = c0 + j;
+            if (e < p.E) {
+              const float v = rank_key(__uint_as_float(r[j]) + s_bias[e]);
+              if (ranks_before(v, e, tv[KMAX - 1], te[KMAX - 1])) {
+                tv[KMAX - 1] = v;
+                te[KMAX - 1] = e;
+#pragma unroll
+                for (int q = KMAX - 1; q > 0; --q) {
+                  if (ranks_before(tv[q], te[q], tv[q - 1], te[q - 1])) {
+                    const float fv = tv[q]; tv[q] = tv[q - 1]; tv[q - 1] = fv;
+                    const int fe = te[q]; te[q] = te[q - 1]; te[q - 1] = fe;
+                  }
+                }
+              }
+            }
+          }
+        }
+      }
+      const float m = tv[0];  // largest logit
+      float denom_all = 0.f;
+      if (EN_T > 0 && p.gate_mode != MOE_GATE_TOPK_SOFTMAX) {
+#pragma unroll
+        for (int e = 0; e < (EN_T > 0 ? EN_T : 1); ++e)
+          if (e < p.E) denom_all += expf(zr[e] - m);
+      } else if (p.gate_mode != MOE_GATE_TOPK_SOFTMAX) {  // softmax over all E: a second pass
+        for (int c0 = 0; c0 < p.EN; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld_32x32b_x16(trow + c0, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int e = c0 + j;
+            if (e < p.E) denom_all += expf(rank_key(__uint_as_float(r[j]) + s_bias[e]) - m);
+          }
+        }
+      }
+      float g[KMAX];
+      float sel = 0.f;
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        g[j] = (j < p.k) ? expf(tv[j] - m) : 0.f;
+        if (p.gate_mode != MOE_GATE_TOPK_SOFTMAX) g[j] = g[j] / denom_all;  // probability
+        sel += g[j];
+      }
+      if (t < p.T) {
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+          if (j < p.k) {
+            const float gj = (p.gate_mode == MOE_GATE_SOFTMAX_TOPK) ? g[j] : g[j] / sel;
+            p.ids[static_cast<size_t>(t) * p.k + j] = te[j];
+            p.gates[static_cast<size_t>(t) * p.k + j] = gj;
+            atomicAdd(&s_hist[te[j]], 1);
+          }
+        }
+      }
+    }
+    epilogue_bar();
+    if (p.tile_hist != nullptr)
+      for (int e = threadIdx.x; e < p.E; e += 128)
+        p.tile_hist[static_cast<size_t>(tile) * p.E + e] = s_hist[e];
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc(tmem_base, p.tmem_cols);
+}
+
+template <int EN_T, int KMAX>
+cudaError_t launch_kmax(const RouteMaps& maps, const RouteParams& p, int grid, int smem,
+                        cudaStream_t s) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<EN_T, KMAX>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         1024 + kRingBudget + 4096);
+    if (e != cudaSuccess) return e;
+    prefer_max_shared(router_tc_kernel<EN_T, KMAX>);
+    configured = true;
+  }
+  return launch_pdl(router_tc_kernel<EN_T, KMAX>, dim3(grid), dim3(kThreads), smem, s, maps, p);
+}
+
+template <int EN_T>
+cudaError_t launch_en(const RouteMaps& maps, const RouteParams& p, int grid, int smem,
+                      cudaStream_t s) {
+  if (p.k <= 1) return launch_kmax<EN_T, 1>(maps, p, grid, smem, s);
+  if (p.k <= 2) return launch_kmax<EN_T, 2>(maps, p, grid, smem, s);
+  if (p.k <= 4) return launch_kmax<EN_T, 4>(maps, p, grid, smem, s);
+  if (p.k <= 8) return launch_kmax<EN_T, 8>(maps, p, grid, smem, s);
+  if (p.k <= 16) return launch_kmax<EN_T, 16>(maps, p, grid, smem, s);
+  return launch_kmax<EN_T, 32>(maps, p, grid, smem, s);
+}
+
+}  // namespace
+
+cudaError_t launch_router_sm100(const moe_config& c, const void* x, const void* w_router,
+                                const float* bias, int32_t* ids, float* gates,
+                                int32_t* tile_hist, int32_t* status, cudaStream_t s) {
+  // Logit columns (MMA N): 16, 32 or 64 when E fits, so the epilogue can keep a token's
+  // logits in registers; otherwise E rounded up to a multiple of 16.
+  const int EN = c.E <= 16 ? 16 : c.E <= 32 ? 32 : c.E <= 64 ? 64 : ((c.E + 15) / 16) * 16;
+  int cols = 32;
+  while (cols < EN) cols *= 2;
+  const int stage_bytes = A_BYTES + EN * BK * 2;
+  int stages = kRingBudget / stage_bytes;
+  if (stages > kMaxStages) stages = kMaxStages;
+  const int k_blocks = c.d / BK;
+  if (stages > k_blocks) stages = k_blocks;
+  RouteMaps maps;
+  if (!encode_2d_box(&maps.x, x, c.d, c.T, kTokens) ||
+      !encode_2d_box(&maps.w, w_router, c.d, c.E, EN))
+    return cudaErrorInvalidValue;
+  RouteParams p{bias, c.T, c.d, c.E, c.k, EN, c.gate_mode, stages, cols,
+                ids, gates, tile_hist, status, kWaitLimitNs};
+  const int grid = (c.T + kTokens - 1) / kTokens;
+  const int smem = 1024 + stages * stage_bytes + 256 + 2 * 256 * 4;
+  if (EN == 16) return launch_en<16>(maps, p, grid, smem, s);
+  if (EN == 32) return launch_en<32>(maps, p, grid, smem, s);
+  if (EN == 64) return launch_en<64>(maps, p, grid, smem, s);
+  return launch_en<0>(maps, p, grid, smem, s);
+}
+
+}  // namespace moe
