@@ -61,7 +61,7 @@ struct ScatterArgs {
   const void* x;
   const int32_t* ids;
   const int32_t* tile_hist;
-  int T, d, k, E, tok_tile, num_tiles, capacity, has_shared;
+  int T, d, k, E, tok_tile, num_tiles, capacity, has_shared, copy_round;
   void* x_packed;
   int32_t* row_token;
   int32_t* route_row;
@@ -71,6 +71,7 @@ struct ScatterArgs {
 };
 
 constexpr int kSubTok = 8;  // tokens packed per CTA
+constexpr size_t kStageBudget = 64 * 1024;  // shared memory staging token rows for the copy
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
@@ -82,6 +83,8 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
   __shared__ int s_off[257];   // segment starts over kept routes
   __shared__ int s_rows[kSubTok][32];
   __shared__ uint32_t s_mask[256 * kWords];  // [E][words]: bit = token of the tile chose e
+  __shared__ __align__(8) uint64_t s_bar;
+  extern __shared__ __align__(128) uint8_t s_stage[];  // copy_round token rows
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t_begin = blockIdx.x * kSubTok;
@@ -177,33 +180,41 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
   }
   __syncthreads();
 
-  // 5. copy: one thread per (token, 16-byte vector), one load and up to k stores; loads of
-  //    kBatch vectors are issued together
+  // 5. copy with the bulk-copy engine: each token row is loaded once into shared memory
+  //    and stored once per kept route (warp 0 issues; the engine moves whole rows)
+  if (warp != 0) return;
+  const uint32_t row_bytes = static_cast<uint32_t>(a.d) * sizeof(T);
+  const int round = a.copy_round;  // token rows staged at a time
   const T* __restrict__ X = static_cast<const T*>(a.x);
   T* __restrict__ XP = static_cast<T*>(a.x_packed);
-  const int nvec = a.d / VEC;
-  const int total = nsub * nvec;
-  for (int i0 = tid; i0 < total; i0 += kThreads * kBatch) {
-    uint4 v[kBatch];
-#pragma unroll
-    for (int q = 0; q < kBatch; ++q) {
-      const int idx = i0 + q * kThreads;
-      if (idx < total) {
-        const int ts = idx / nvec, c = idx - ts * nvec;
-        v[q] = ld_vec(X + static_cast<size_t>(t_begin + ts) * a.d + c * VEC);
-      }
+  if (lane == 0) {
+    mbar_init(&s_bar, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  uint32_t phase = 0;
+  for (int r0 = 0; r0 < nsub; r0 += round) {
+    const int nr = min(round, nsub - r0);
+    int ok = 1;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&s_bar, nr * row_bytes);
+      for (int i = 0; i < nr; ++i)
+        bulk_load(s_stage + i * row_bytes, X + static_cast<size_t>(t_begin + r0 + i) * a.d, row_bytes,
+                  &s_bar);
+      ok = mbar_wait_bounded(&s_bar, phase, nullptr, kWaitLimitNs, a.status);
+      if (!ok) mbar_wait_bounded(&s_bar, phase, nullptr, kWaitLimitNs, a.status);  // drain
     }
-#pragma unroll
-    for (int q = 0; q < kBatch; ++q) {
-      const int idx = i0 + q * kThreads;
-      if (idx < total) {
-        const int ts = idx / nvec, c = idx - ts * nvec;
-        for (int j = 0; j < k; ++j) {
-          const int r = s_rows[ts][j];
-          if (r >= 0) st_vec(XP + static_cast<size_t>(r) * a.d + c * VEC, v[q]);
-        }
-      }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    phase ^= 1u;
+    if (!ok) return;
+    for (int q = lane; q < nr * k; q += 32) {
+      const int i = q / k, j = q - i * k;
+      const int r = s_rows[r0 + i][j];
+      if (r >= 0) bulk_store(XP + static_cast<size_t>(r) * a.d, s_stage + i * row_bytes, row_bytes);
     }
+    bulk_commit();
+    bulk_wait_all();  // the stage is reused next round; the rows are written before exit
+    __syncwarp();
   }
 }
 
@@ -227,18 +238,26 @@ cudaError_t launch_dispatch_scatter(const moe_config& c, const void* x, const in
                                     int32_t* row_token, int32_t* route_row, int32_t* offsets,
                                     int32_t* demand, int32_t* status, cudaStream_t s) {
   const int grid = (c.T + kSubTok - 1) / kSubTok;
+  const size_t row_bytes = static_cast<size_t>(c.d) * (c.dtype == MOE_BF16 ? 2 : 4);
+  int round = static_cast<int>(kStageBudget / row_bytes);
+  round = round < 1 ? 1 : (round > kSubTok ? kSubTok : round);
   ScatterArgs a{x, ids, tile_hist, c.T, c.d, c.k, c.E, kHistTile, num_tiles_for(c.T, c.E),
-                c.capacity, c.has_shared, x_packed, row_token, route_row, offsets, demand,
+                c.capacity, c.has_shared, round, x_packed, row_token, route_row, offsets, demand,
                 status};
+  const size_t smem = static_cast<size_t>(round) * row_bytes;
   static bool configured = false;
   if (!configured) {
     prefer_max_shared(scatter_kernel<__nv_bfloat16>);
     prefer_max_shared(scatter_kernel<float>);
+    cudaFuncSetAttribute(scatter_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(kStageBudget));
+    cudaFuncSetAttribute(scatter_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(kStageBudget));
     configured = true;
   }
   if (c.dtype == MOE_BF16)
-    return launch_pdl(scatter_kernel<__nv_bfloat16>, dim3(grid), dim3(kThreads), 0, s, a);
-  return launch_pdl(scatter_kernel<float>, dim3(grid), dim3(kThreads), 0, s, a);
+    return launch_pdl(scatter_kernel<__nv_bfloat16>, dim3(grid), dim3(kThreads), smem, s, a);
+  return launch_pdl(scatter_kernel<float>, dim3(grid), dim3(kThreads), smem, s, a);
 }
 
 }  // namespace moe
