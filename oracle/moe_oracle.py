@@ -365,3 +365,33 @@ def drop_count(demand, C: int | None) -> int:
     if C is None:
         return 0
     return int(sum(max(0, int(D) - C) for D in demand))
+
+
+def routing_stats(x, w_router, logit_bias, k: int, C: int | None, alpha: float = 1e-2,
+                  ids=None):
+    """Routing statistics of one layer call, in float64.
+
+    f_e   fraction of routes dispatched to expert e before capacity (demand_e / (T k));
+          [MoE-L] section 4 defines f_i as the fraction dispatched to expert i for top-1;
+          with top-k the routes are counted, so that sum_e f_e = 1 as in the top-1 case.
+    P_e   mean over tokens of the full softmax probability of expert e ([MoE-L] section 4,
+          "the mean routing probability").
+    aux   alpha * E * sum_e f_e P_e ([MoE-L] section 4; alpha = 1e-2 as reported there).
+    I     max_e demand_e / mean_e demand_e on pre-capacity demand ([MoE-AEV] Load imbalance).
+    drop  dropped routes / (T k); padding: empty slots / (E C) of the capacity buffer
+          ([MoE-S19] Worked case: 20 slots, 15 used, 25% padding); 0 when dropless or
+          C = 0 (no slots).
+    Returns a dict with those entries and kept (the number of kept routes).
+    """
+    z = router_logits(x, w_router, logit_bias)
+    T, E = z.shape
+    if ids is None:
+        ids = top_k(z, k)
+    d = dispatch(ids, E, C)
+    demand = d["demand"].astype(np.float64)
+    f = demand / (T * k)
+    P = softmax(z).mean(axis=0)
+    kept = int(d["kept"].sum())
+    return dict(f=f, P=P, aux=alpha * E * float(np.sum(f * P)), imbalance=imbalance(demand),
+                drop_rate=(T * k - kept) / (T * k),
+                padding_rate=(0.0 if not C else (E * C - kept) / (E * C)), kept=kept)

@@ -379,3 +379,64 @@ def test_stack_route_count_and_residual():
     x2 = O.round_to_bf16(y2)
     y3, _ = O.moe_layer(x2, layers[2], 2, O.GATE_TOPK_SOFTMAX, add_residual=True)
     assert np.array_equal(xL, O.round_to_bf16(y3))
+
+
+# ---------------------------------------------------------------- routing statistics
+
+def test_routing_stats_worked_case(golden):
+    """[S19] worked case: demand 6/4/3/3, C = 5, one drop, 15 of 20 slots used (25% padding)."""
+    g = golden("capacity_worked_case.json")
+    ids = np.array(g["assignments"])
+    T, E, k = g["T"], g["E"], g["k"]
+    rng = np.random.default_rng(12)
+    x, w = rng.normal(size=(T, 8)), rng.normal(size=(E, 8))
+    st = O.routing_stats(x, w, None, k, g["C"], ids=ids)
+    assert st["kept"] == g["filled"] == 15
+    assert st["padding_rate"] == (g["slots"] - g["filled"]) / g["slots"] == 0.25
+    assert st["drop_rate"] == 1 / 16
+    assert st["imbalance"] == 6 / 4
+    assert np.allclose(st["f"], np.array(g["demand"]) / 16, rtol=0, atol=0)
+    assert abs(st["P"].sum() - 1) < 1e-12
+
+
+def test_aux_loss_closed_forms():
+    """Uniform routing gives aux = alpha; a collapsed router gives aux -> alpha * E."""
+    T, E, d = 64, 8, 4
+    x = np.zeros((T, d))
+    w = np.zeros((E, d))
+    ids = np.array([[t % E] for t in range(T)])          # every expert gets T/E routes
+    st = O.routing_stats(x, w, None, 1, None, alpha=0.01, ids=ids)
+    assert np.allclose(st["f"], 1 / E) and np.allclose(st["P"], 1 / E)
+    assert abs(st["aux"] - 0.01) < 1e-15
+    bias = np.zeros(E)
+    bias[0] = 60.0                                        # softmax ~ one-hot on expert 0
+    st = O.routing_stats(np.ones((T, d)), np.zeros((E, d)), bias, 1, None, alpha=0.01)
+    assert st["f"][0] == 1.0 and st["P"][0] > 1 - 1e-12
+    assert abs(st["aux"] - 0.01 * E) < 1e-12
+    assert st["imbalance"] == E / 1
+
+
+def test_routing_stats_drop_and_padding_brute_force():
+    """Drop and padding rates against a slot-by-slot count, including C = 0 (no slots)."""
+    rng = np.random.default_rng(3)
+    T, E, k, d = 50, 6, 2, 5
+    x, w = rng.normal(size=(T, d)), rng.normal(size=(E, d))
+    ids = O.top_k(O.router_logits(x, w), k)
+    for C in (None, 0, 3, 17, 100):
+        st = O.routing_stats(x, w, None, k, C, ids=ids)
+        used = [0] * E
+        kept = 0
+        for t in range(T):                 # arrival order = token order
+            for j in range(k):
+                e = int(ids[t, j])
+                if C is None or used[e] < C:
+                    used[e] += 1
+                    kept += 1
+        assert st["kept"] == kept
+        assert st["drop_rate"] == (T * k - kept) / (T * k)
+        assert st["padding_rate"] == (0.0 if not C else sum(C - u for u in used) / (E * C))
+        # P: the mean of the full softmax, one token at a time
+        z = O.router_logits(x, w)
+        P = sum(np.exp(z[t] - z[t].max()) / np.exp(z[t] - z[t].max()).sum() for t in range(T)) / T
+        assert np.allclose(st["P"], P, rtol=1e-13, atol=0)
+        assert abs(st["aux"] - 1e-2 * E * sum(st["f"][e] * P[e] for e in range(E))) < 1e-15
