@@ -78,6 +78,8 @@ typedef struct {
   int32_t capacity;     /* < 0: dropless; else C >= 0 rows per expert (see moe_capacity) */
   int32_t has_shared;   /* 1: one always-on shared expert, gate 1, never dropped          */
   int32_t add_residual; /* 1: y = x + MoE(x)                                              */
+  int32_t stats;        /* 1: the router also sums each token's full softmax per token
+                         *    tile into the workspace, for moe_routing_stats; 0: off     */
 } moe_config;
 /* Supported shapes (else MOE_ERR_UNSUPPORTED): bf16 needs d % 128 == 0 and
  * d_ff % 128 == 0; fp32 needs d % 4 == 0 and d_ff % 4 == 0.                            */
@@ -208,6 +210,41 @@ moe_status moe_dispatch_noalloc(const moe_config* cfg, const void* x, const int3
                                 void* x_packed, int32_t* row_token, int32_t* route_row,
                                 int32_t* offsets, int32_t* demand, int32_t* status,
                                 moe_stream_t stream);
+
+/* Routing statistics of one layer call, written by moe_routing_stats (device memory). */
+typedef struct {
+  float aux_loss;        /* alpha * E * sum_e f_e * P_e                                      */
+  float imbalance;       /* max_e demand_e / mean_e demand_e; 0 when no route is valid       */
+  float drop_rate;       /* (T*k - kept) / (T*k)                                             */
+  float padding_rate;    /* (E*C - kept) / (E*C) with capacity C > 0; 0 when dropless, C = 0 */
+  int32_t kept;          /* kept routes R = offsets[E]                                       */
+  int32_t dropped;       /* T*k - R                                                          */
+  int32_t max_demand;    /* max_e demand_e                                                   */
+  int32_t busiest_expert;/* lowest e with demand_e = max_demand                              */
+} moe_routing_summary;
+
+/* Routing statistics of the last routed call on `ws`: the load-balancing terms and the
+ * capacity outcome ("Mixture of Experts: Routing, Dispatch, and Load Balancing", section 4:
+ * loss_aux = alpha * N * sum_i f_i P_i with f_i the fraction of tokens dispatched to
+ * expert i and P_i the mean router probability; "Mixture-of-experts routing", Load
+ * imbalance: I = max_e D_e / mean_e D_e; "Mixture-of-Experts: routing and capacity",
+ * Worked case: drops and empty slots of the E x C buffer).
+ *   f_e = demand_e / (T k): routes asking for e before capacity (with top-k each route
+ *         counts once, so sum_e f_e = 1 when every id is valid).
+ *   P_e = (1/T) sum_t softmax(z_t)_e over all E experts, whatever the gate mode.
+ * Requires cfg->stats = 1 for the moe_route or moe_forward call that routed on this
+ * workspace (its per-tile probability sums are read from `ws`; MOE_ERR_INVALID if
+ * cfg->stats is 0).  Sums run in a fixed order (fp32 within a 128-token tile, fp64 across
+ * tiles), so repeated calls give identical bits.
+ *   demand   [E] int32, offsets [E+2] int32: from moe_dispatch, or moe_forward's
+ *            demand_out / offsets_out.  NULL: the copies moe_forward keeps in `ws` when its
+ *            own *_out argument was NULL.
+ *   alpha    weight of the auxiliary value (1e-2 in the Switch Transformer setup).
+ *   f, P     [E] fp32 (out, device) or NULL.     summary: one moe_routing_summary (out,
+ *            device), required.                                                        */
+moe_status moe_routing_stats(const moe_config* cfg, const int32_t* demand,
+                             const int32_t* offsets, float alpha, float* f, float* P,
+                             moe_routing_summary* summary, void* ws, moe_stream_t stream);
 
 /* Static string for a status code. */
 const char* moe_status_string(moe_status s);

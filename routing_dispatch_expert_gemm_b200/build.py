@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_PATH = os.path.join(HERE, "libmoe.so")
 
-SOURCES = ["api.cu", "route.cu", "route_sm100.cu", "dispatch.cu", "gemm_simt.cu",
+SOURCES = ["api.cu", "route.cu", "route_sm100.cu", "dispatch.cu", "gemm_simt.cu", "stats.cu",
            "gemm_sm100.cu", "combine.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",

@@ -3,6 +3,7 @@
 // behaviour, in include/moe.h.
 #include <algorithm>
 #include <climits>
+#include <cmath>
 
 #include "common.cuh"
 #include "internal.h"
@@ -11,7 +12,7 @@ using namespace moe;
 
 namespace {
 
-constexpr int32_t kAbiVersion = 1;
+constexpr int32_t kAbiVersion = 2;
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
@@ -22,7 +23,8 @@ moe_status validate(const moe_config* c) {
   if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID;
   if (c->gate_mode < MOE_GATE_SOFTMAX_TOPK || c->gate_mode > MOE_GATE_TOPK_SOFTMAX)
     return MOE_ERR_INVALID;
-  if ((c->has_shared != 0 && c->has_shared != 1) || (c->add_residual != 0 && c->add_residual != 1))
+  if ((c->has_shared != 0 && c->has_shared != 1) || (c->add_residual != 0 && c->add_residual != 1) ||
+      (c->stats != 0 && c->stats != 1))
     return MOE_ERR_INVALID;
   if (c->E > 256 || c->k > 32) return MOE_ERR_UNSUPPORTED;
   if (c->T > (1 << 24) || static_cast<int64_t>(c->T) * c->k > (INT_MAX / 2)) return MOE_ERR_UNSUPPORTED;
@@ -41,7 +43,8 @@ int64_t max_rows(const moe_config& c) {
 }
 
 struct Layout {
-  size_t tile_hist, ids, gates, route_row, row_token, offsets, demand, x_packed, h, y_packed;
+  size_t tile_hist, tile_psum, stats_partial, ids, gates, route_row, row_token, offsets, demand;
+  size_t x_packed, h, y_packed;
   size_t scratch_end, total;
   int64_t rmax, rows_h;
 };
@@ -59,6 +62,9 @@ Layout layout_of(const moe_config& c) {
   L.rmax = max_rows(c);
   L.rows_h = L.rmax + (c.has_shared ? c.T : 0);
   L.tile_hist = take(static_cast<size_t>(num_tiles_for(c.T, c.E)) * c.E * 4);
+  // Routing statistics (only with cfg.stats): per-tile probability sums and fp64 partials.
+  L.tile_psum = c.stats ? take(static_cast<size_t>(num_tiles_for(c.T, c.E)) * c.E * 4) : 0;
+  L.stats_partial = c.stats ? take(static_cast<size_t>(kStatsMaxBlocks) * c.E * 8) : 0;
   L.scratch_end = off;
   L.ids = take(Tk * 4);
   L.gates = take(Tk * 4);
@@ -115,6 +121,7 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
   const Layout L = layout_of(c);
   int32_t* status = static_cast<int32_t*>(ws);
   int32_t* hist = reinterpret_cast<int32_t*>(at(ws, L.tile_hist));
+  float* psum = c.stats ? reinterpret_cast<float*>(at(ws, L.tile_psum)) : nullptr;
   int32_t* ids = ids_out ? ids_out : reinterpret_cast<int32_t*>(at(ws, L.ids));
   float* gates = gates_out ? gates_out : reinterpret_cast<float*>(at(ws, L.gates));
   int32_t* demand = demand_out ? demand_out : reinterpret_cast<int32_t*>(at(ws, L.demand));
@@ -126,7 +133,8 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
   void* y_packed = at(ws, L.y_packed);
 
   MOE_TRY(record(ev, 0, stream));
-  MOE_TRY(cuda_status(launch_router(c, x, w_router, logit_bias, ids, gates, hist, status, stream)));
+  MOE_TRY(cuda_status(
+      launch_router(c, x, w_router, logit_bias, ids, gates, hist, psum, status, stream)));
   MOE_TRY(record(ev, 1, stream));
   MOE_TRY(cuda_status(launch_dispatch_scatter(c, x, ids, hist, x_packed, row_token, route_row,
                                               offsets, demand, status, stream)));
@@ -188,9 +196,10 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router,
   MOE_TRY(check_ws(ws));
   if (!x || !w_router || !ids || !gates) return MOE_ERR_INVALID;
   const Layout L = layout_of(*cfg);
-  return cuda_status(launch_router(*cfg, x, w_router, logit_bias, ids, gates,
-                                   reinterpret_cast<int32_t*>(at(ws, L.tile_hist)),
-                                   static_cast<int32_t*>(ws), stream));
+  return cuda_status(launch_router(
+      *cfg, x, w_router, logit_bias, ids, gates, reinterpret_cast<int32_t*>(at(ws, L.tile_hist)),
+      cfg->stats ? reinterpret_cast<float*>(at(ws, L.tile_psum)) : nullptr,
+      static_cast<int32_t*>(ws), stream));
 }
 
 moe_status moe_dispatch(const moe_config* cfg, const void* x, const int32_t* ids,
@@ -257,6 +266,21 @@ moe_status moe_forward_profiled(const moe_config* cfg, const void* x, const void
   return forward_impl(cfg, x, w_router, logit_bias, w_gate, w_up, w_down, shared_gate, shared_up,
                       shared_down, y, ids_out, gates_out, demand_out, offsets_out, events, ws,
                       stream);
+}
+
+moe_status moe_routing_stats(const moe_config* cfg, const int32_t* demand,
+                             const int32_t* offsets, float alpha, float* f, float* P,
+                             moe_routing_summary* summary, void* ws, moe_stream_t stream) {
+  MOE_TRY(validate(cfg));
+  MOE_TRY(check_ws(ws));
+  if (!cfg->stats || summary == nullptr || !std::isfinite(alpha)) return MOE_ERR_INVALID;
+  const Layout L = layout_of(*cfg);
+  const int32_t* dem = demand ? demand : reinterpret_cast<const int32_t*>(at(ws, L.demand));
+  const int32_t* off = offsets ? offsets : reinterpret_cast<const int32_t*>(at(ws, L.offsets));
+  return cuda_status(launch_routing_stats(
+      *cfg, reinterpret_cast<const float*>(at(ws, L.tile_psum)), dem, off, alpha,
+      reinterpret_cast<double*>(at(ws, L.stats_partial)),
+      reinterpret_cast<unsigned int*>(at(ws, kWsStatsCounterOffset)), f, P, summary, stream));
 }
 
 moe_status moe_get_device_status(void* ws, moe_stream_t stream, int32_t clear,

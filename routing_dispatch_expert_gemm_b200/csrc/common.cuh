@@ -14,6 +14,8 @@ namespace moe {
 // Workspace header: the device status word lives at byte 0 of every workspace.
 // ---------------------------------------------------------------------------------
 constexpr size_t kWsHeaderBytes = 256;
+// Byte offset, in the header, of the ticket counter of the routing-statistics kernel.
+constexpr size_t kWsStatsCounterOffset = 64;
 
 // First error wins; later errors do not overwrite it.
 __device__ __forceinline__ void record_status(int32_t* status, int32_t code) {

@@ -14,14 +14,25 @@ constexpr int kHistTile = 128;
 inline int tok_tile_for(int /*T*/, int /*E*/) { return kHistTile; }
 inline int num_tiles_for(int T, int /*E*/) { return (T + kHistTile - 1) / kHistTile; }
 
+// tile_psum (may be null): [num_tiles, E] fp32, the sum over each token tile of every
+// token's full softmax, for the routing statistics.
 cudaError_t launch_router(const moe_config& c, const void* x, const void* w_router,
                           const float* bias, int32_t* ids, float* gates, int32_t* tile_hist,
-                          int32_t* status, cudaStream_t s);
+                          float* tile_psum, int32_t* status, cudaStream_t s);
 
 // bf16 router on tensor cores (route_sm100.cu); the fp32 router runs on CUDA cores.
 cudaError_t launch_router_sm100(const moe_config& c, const void* x, const void* w_router,
                                 const float* bias, int32_t* ids, float* gates,
-                                int32_t* tile_hist, int32_t* status, cudaStream_t s);
+                                int32_t* tile_hist, float* tile_psum, int32_t* status,
+                                cudaStream_t s);
+
+// Routing statistics from the per-tile probability sums and the dispatch counts.
+// partial: [kStatsMaxBlocks, E] fp64 scratch; counter: zero before the call, left zero.
+constexpr int kStatsMaxBlocks = 148;
+cudaError_t launch_routing_stats(const moe_config& c, const float* tile_psum,
+                                 const int32_t* demand, const int32_t* offsets, float alpha,
+                                 double* partial, unsigned int* counter, float* f, float* P,
+                                 moe_routing_summary* out, cudaStream_t s);
 
 cudaError_t launch_dispatch_hist(const moe_config& c, const int32_t* ids, int32_t* tile_hist,
                                  int32_t* status, cudaStream_t s);

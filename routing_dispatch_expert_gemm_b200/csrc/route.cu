@@ -37,6 +37,7 @@ struct RouterArgs {
   int32_t* ids;
   float* gates;
   int32_t* tile_hist;
+  float* tile_psum;  // null: no routing statistics
 };
 
 // NaN logits rank as -inf so that k valid experts are always selected.
@@ -75,6 +76,7 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(RouterArgs a) {
   constexpr int NP = (EP == 32) ? 8 : 1;  // passes over experts (E <= 256)
   extern __shared__ uint4 s_w[];          // [EP][dc / VEC] vectors
   __shared__ int s_hist[256];
+  __shared__ float s_psum[8][256];  // per-warp running sums of full-softmax probabilities
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile = blockIdx.x;
@@ -86,6 +88,8 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(RouterArgs a) {
   const Tin* __restrict__ W = static_cast<const Tin*>(a.w);
 
   for (int e = tid; e < a.E; e += kThreads) s_hist[e] = 0;
+  if (a.tile_psum != nullptr)
+    for (int i = tid; i < 8 * 256; i += kThreads) s_psum[i >> 8][i & 255] = 0.f;
   pdl_trigger();
   pdl_wait();
 
@@ -192,17 +196,32 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(RouterArgs a) {
       const float m = __shfl_sync(0xffffffffu, sel_z, 0);  // largest selected logit
       const float ej = (lane < a.k) ? expf(sel_z - m) : 0.f;
       float g;
-      if (a.gate_mode == MOE_GATE_TOPK_SOFTMAX) {
-        g = ej / warp_sum(ej);
-      } else {
+      float denom_all = 0.f;
+      if (a.gate_mode != MOE_GATE_TOPK_SOFTMAX || a.tile_psum != nullptr) {
         float local = 0.f;
 #pragma unroll
         for (int p = 0; p < NP; ++p) {
           const int ge = p * EP + lane;
           if (p < npass && lane < EP && ge < a.E) local += expf(rank_key(zl[i][p]) - m);
         }
-        const float pj = ej / warp_sum(local);
+        denom_all = warp_sum(local);
+      }
+      if (a.gate_mode == MOE_GATE_TOPK_SOFTMAX) {
+        g = ej / warp_sum(ej);
+      } else {
+        const float pj = ej / denom_all;
         g = (a.gate_mode == MOE_GATE_SOFTMAX_TOPK) ? pj : pj / warp_sum(pj);
+      }
+      if (a.tile_psum != nullptr) {
+        // Routing statistics: this warp adds its tokens' full softmax in token order;
+        // expert ge belongs to exactly one lane, so the per-warp sums are race-free.
+        const float inv = 1.f / denom_all;
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+          const int ge = p * EP + lane;
+          if (p < npass && lane < EP && ge < a.E)
+            s_psum[warp][ge] += expf(rank_key(zl[i][p]) - m) * inv;
+        }
       }
       if (lane < a.k) {
         a.ids[static_cast<size_t>(t) * a.k + lane] = sel_e;
@@ -215,6 +234,13 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(RouterArgs a) {
   if (a.tile_hist != nullptr)
     for (int e = tid; e < a.E; e += kThreads)
       a.tile_hist[static_cast<size_t>(tile) * a.E + e] = s_hist[e];
+  if (a.tile_psum != nullptr)
+    for (int e = tid; e < a.E; e += kThreads) {
+      float v = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) v += s_psum[w][e];
+      a.tile_psum[static_cast<size_t>(tile) * a.E + e] = v;
+    }
 }
 
 template <typename Tin, int EP>
@@ -254,11 +280,11 @@ cudaError_t launch_typed(RouterArgs a, cudaStream_t s) {
 
 cudaError_t launch_router(const moe_config& c, const void* x, const void* w_router,
                           const float* bias, int32_t* ids, float* gates, int32_t* tile_hist,
-                          int32_t* status, cudaStream_t s) {
+                          float* tile_psum, int32_t* status, cudaStream_t s) {
   if (c.dtype == MOE_BF16)
-    return launch_router_sm100(c, x, w_router, bias, ids, gates, tile_hist, status, s);
+    return launch_router_sm100(c, x, w_router, bias, ids, gates, tile_hist, tile_psum, status, s);
   RouterArgs a{x, w_router, bias, c.T, c.d, c.E, c.k, c.gate_mode, kHistTile, 0,
-               ids, gates, tile_hist};
+               ids, gates, tile_hist, tile_psum};
   return launch_typed<float>(a, s);
 }
 

@@ -51,6 +51,7 @@ struct RouteParams {
   int32_t* ids;
   float* gates;
   int32_t* tile_hist;
+  float* tile_psum;  // null: no routing statistics
   int32_t* status;
   int64_t limit_ns;
 };
@@ -74,6 +75,14 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* r) 
 }
 
 __device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Sum over the warp's 32 lanes.  The butterfly pairs the same two partial sums on both
+// lanes of each exchange, so every lane ends with identical bits.
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) v += __shfl_xor_sync(0xffffffffu, v, s);
+  return v;
+}
 
 // Top-k of one token's logits z[0..NV) held in registers: k rounds of a tournament
 // (binary-tree arg-max).  At every node the left child covers lower expert indices, so
@@ -132,6 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* s_bias = reinterpret_cast<float*>(ctl + 256);
   int* s_hist = reinterpret_cast<int*>(ctl + 256 + 256 * 4);
+  float* s_psum = reinterpret_cast<float*>(ctl + 256 + 2 * 256 * 4);  // [4 warps][256]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = blockIdx.x;
@@ -158,6 +168,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     s_bias[e] = (e < p.E && p.bias != nullptr) ? __ldg(p.bias + e) : 0.f;
     s_hist[e] = 0;
   }
+  if (p.tile_psum != nullptr)
+    for (int i = threadIdx.x; i < 4 * 256; i += kThreads) s_psum[i] = 0.f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -264,12 +276,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       const float m = tv[0];  // largest logit
+      const bool want_all = p.gate_mode != MOE_GATE_TOPK_SOFTMAX || p.tile_psum != nullptr;
       float denom_all = 0.f;
-      if (EN_T > 0 && p.gate_mode != MOE_GATE_TOPK_SOFTMAX) {
+      if (EN_T > 0 && want_all) {
 #pragma unroll
         for (int e = 0; e < (EN_T > 0 ? EN_T : 1); ++e)
           if (e < p.E) denom_all += expf(zr[e] - m);
-      } else if (p.gate_mode != MOE_GATE_TOPK_SOFTMAX) {  // softmax over all E: a second pass
+      } else if (want_all) {  // softmax over all E: a second pass
         for (int c0 = 0; c0 < p.EN; c0 += 16) {
           uint32_t r[16];
           tmem_ld_32x32b_x16(trow + c0, r);
@@ -300,11 +313,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      if (p.tile_psum != nullptr) {
+        // Routing statistics: every token's full softmax, summed over the warp's 32
+        // tokens one expert at a time (tokens past T contribute zero).
+        const float inv = (t < p.T) ? 1.f / denom_all : 0.f;
+        if constexpr (EN_T > 0) {
+#pragma unroll
+          for (int e = 0; e < EN_T; ++e) {
+            const float v = warp_sum(expf(zr[e] - m) * inv);  // zr = -inf past E
+            if (lane == (e & 31) && e < p.E) s_psum[warp * 256 + e] = v;
+          }
+        } else {
+          for (int c0 = 0; c0 < p.EN; c0 += 16) {
+            uint32_t r[16];
+            tmem_ld_32x32b_x16(trow + c0, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int e = c0 + j;
+              const float z = (e < p.E) ? rank_key(__uint_as_float(r[j]) + s_bias[e]) : -INFINITY;
+              const float v = warp_sum(expf(z - m) * inv);
+              if (lane == (e & 31) && e < p.E) s_psum[warp * 256 + e] = v;
+            }
+          }
+        }
+      }
     }
     epilogue_bar();
     if (p.tile_hist != nullptr)
       for (int e = threadIdx.x; e < p.E; e += 128)
         p.tile_hist[static_cast<size_t>(tile) * p.E + e] = s_hist[e];
+    if (p.tile_psum != nullptr)
+      for (int e = threadIdx.x; e < p.E; e += 128)
+        p.tile_psum[static_cast<size_t>(tile) * p.E + e] =
+            ((s_psum[e] + s_psum[256 + e]) + s_psum[512 + e]) + s_psum[768 + e];
   }
 
   tc_fence_before();
@@ -320,7 +362,7 @@ cudaError_t launch_kmax(const RouteMaps& maps, const RouteParams& p, int grid, i
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<EN_T, KMAX>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         1024 + kRingBudget + 4096);
+                                         1024 + kRingBudget + 8192);
     if (e != cudaSuccess) return e;
     prefer_max_shared(router_tc_kernel<EN_T, KMAX>);
     configured = true;
@@ -343,7 +385,8 @@ cudaError_t launch_en(const RouteMaps& maps, const RouteParams& p, int grid, int
 
 cudaError_t launch_router_sm100(const moe_config& c, const void* x, const void* w_router,
                                 const float* bias, int32_t* ids, float* gates,
-                                int32_t* tile_hist, int32_t* status, cudaStream_t s) {
+                                int32_t* tile_hist, float* tile_psum, int32_t* status,
+                                cudaStream_t s) {
   // Logit columns (MMA N): 16, 32 or 64 when E fits, so the epilogue can keep a token's
   // logits in registers; otherwise E rounded up to a multiple of 16.
   const int EN = c.E <= 16 ? 16 : c.E <= 32 ? 32 : c.E <= 64 ? 64 : ((c.E + 15) / 16) * 16;
@@ -359,9 +402,9 @@ cudaError_t launch_router_sm100(const moe_config& c, const void* x, const void* 
       !encode_2d_box(&maps.w, w_router, c.d, c.E, EN))
     return cudaErrorInvalidValue;
   RouteParams p{bias, c.T, c.d, c.E, c.k, EN, c.gate_mode, stages, cols,
-                ids, gates, tile_hist, status, kWaitLimitNs};
+                ids, gates, tile_hist, tile_psum, status, kWaitLimitNs};
   const int grid = (c.T + kTokens - 1) / kTokens;
-  const int smem = 1024 + stages * stage_bytes + 256 + 2 * 256 * 4;
+  const int smem = 1024 + stages * stage_bytes + 256 + 2 * 256 * 4 + (tile_psum ? 4 * 256 * 4 : 0);
   if (EN == 16) return launch_en<16>(maps, p, grid, smem, s);
   if (EN == 32) return launch_en<32>(maps, p, grid, smem, s);
   if (EN == 64) return launch_en<64>(maps, p, grid, smem, s);

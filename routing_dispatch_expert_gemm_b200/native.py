@@ -13,6 +13,7 @@ import os
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
 
 MOE_OK = 0
+ABI_VERSION = 2  # moe_abi_version() of the library this binding mirrors
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID", 2: "MOE_ERR_UNSUPPORTED",
                 3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_BAD_EXPERT_ID",
                 6: "MOE_ERR_TIMEOUT"}
@@ -23,7 +24,8 @@ GATE_MODES = {"softmax_topk": 0, "softmax_topk_renorm": 1, "topk_softmax": 2}
 EXPORTS = ("moe_capacity", "moe_max_rows", "moe_workspace_bytes", "moe_workspace_init",
            "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_forward_profiled", "moe_get_device_status", "moe_debug_bounded_wait",
-           "moe_dispatch_noalloc", "moe_status_string", "moe_abi_version")
+           "moe_dispatch_noalloc", "moe_routing_stats", "moe_status_string",
+           "moe_abi_version")
 
 
 class MoeError(RuntimeError):
@@ -35,17 +37,32 @@ class MoeError(RuntimeError):
 class MoeConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("T", "d", "E", "k", "d_ff", "dtype", "gate_mode", "capacity",
-                 "has_shared", "add_residual")]
+                 "has_shared", "add_residual", "stats")]
 
     def __repr__(self):
         return "MoeConfig(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
 
 
 def make_config(T, d, E, k, d_ff, dtype="bf16", gate_mode="topk_softmax", capacity=-1,
-                has_shared=False, add_residual=False) -> MoeConfig:
+                has_shared=False, add_residual=False, stats=False) -> MoeConfig:
     return MoeConfig(int(T), int(d), int(E), int(k), int(d_ff), DTYPES[dtype],
                      GATE_MODES[gate_mode], int(capacity), int(bool(has_shared)),
-                     int(bool(add_residual)))
+                     int(bool(add_residual)), int(bool(stats)))
+
+
+class MoeRoutingSummary(ctypes.Structure):
+    """moe_routing_summary; moe_routing_stats writes one into device memory."""
+    _fields_ = [("aux_loss", ctypes.c_float), ("imbalance", ctypes.c_float),
+                ("drop_rate", ctypes.c_float), ("padding_rate", ctypes.c_float),
+                ("kept", ctypes.c_int32), ("dropped", ctypes.c_int32),
+                ("max_demand", ctypes.c_int32), ("busiest_expert", ctypes.c_int32)]
+
+
+def summary_dict(buf) -> dict:
+    """Decode a moe_routing_summary copied to the host (bytes, or a uint8 tensor/array)."""
+    raw = bytes(buf.cpu().numpy().tobytes()) if hasattr(buf, "cpu") else bytes(buf)
+    s = MoeRoutingSummary.from_buffer_copy(raw[:ctypes.sizeof(MoeRoutingSummary)])
+    return {n: getattr(s, n) for n, _ in s._fields_}
 
 
 _lib = None
@@ -76,12 +93,16 @@ def lib() -> ctypes.CDLL:
             "moe_get_device_status": (_I32, [_P, _P, _I32, ctypes.POINTER(_I32)]),
             "moe_debug_bounded_wait": (_I32, [_P, ctypes.c_int64, _P]),
             "moe_dispatch_noalloc": (_I32, [_CFG] + [_P] * 8 + [_P]),
+            "moe_routing_stats": (_I32, [_CFG, _P, _P, ctypes.c_float, _P, _P, _P, _P, _P]),
             "moe_status_string": (ctypes.c_char_p, [_I32]),
             "moe_abi_version": (_I32, []),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
             f.restype, f.argtypes = res, args
+        if L.moe_abi_version() != ABI_VERSION:
+            raise ImportError(f"{LIB_PATH} has ABI version {L.moe_abi_version()}, the binding "
+                              f"expects {ABI_VERSION}: rebuild the library")
         _lib = L
     return _lib
 
@@ -204,6 +225,13 @@ def moe_dispatch_noalloc(cfg, x, ids, x_packed, row_token, route_row, offsets, d
                                       _ptr(row_token), _ptr(route_row), _ptr(offsets),
                                       _ptr(demand), _ptr(status), _stream(stream)),
            "moe_dispatch_noalloc")
+
+
+def moe_routing_stats(cfg, demand, offsets, alpha, f, P, summary, ws, stream=None):
+    """``summary``: a device uint8 tensor of at least 32 bytes (decode with summary_dict)."""
+    _check(lib().moe_routing_stats(ctypes.byref(cfg), _ptr(demand), _ptr(offsets),
+                                   float(alpha), _ptr(f), _ptr(P), _ptr(summary), _ptr(ws),
+                                   _stream(stream)), "moe_routing_stats")
 
 
 def workspace(cfg: MoeConfig, device="cuda"):

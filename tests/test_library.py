@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(native):
     lib = ctypes.CDLL(native.LIB_PATH)
     for name in declared:
         assert hasattr(lib, name), name
-    assert native.moe_abi_version() == 1
+    assert native.moe_abi_version() == native.ABI_VERSION == 2
 
 
 def test_library_is_sm100a_build(native):
@@ -104,3 +104,27 @@ def test_errors_return_before_any_launch(native):
                            None, None, None, None, None, None, 4096, None) == 1
     assert lib.moe_debug_bounded_wait(4096, 10, None) == 1
     assert native.moe_status_string(6).startswith("a bounded")
+
+
+def test_routing_stats_arguments(native):
+    lib = native.lib()
+    fake = 1 << 20  # never dereferenced: validation fails first
+    off = native.make_config(8, 128, 4, 2, 128)
+    on = native.make_config(8, 128, 4, 2, 128, stats=True)
+    # the statistics need the router's per-tile sums: cfg.stats = 0 is rejected
+    assert lib.moe_routing_stats(ctypes.byref(off), fake, fake, 0.01, None, None, fake, 4096,
+                                 None) == 1
+    assert lib.moe_routing_stats(ctypes.byref(on), fake, fake, 0.01, None, None, None, 4096,
+                                 None) == 1                              # summary required
+    assert lib.moe_routing_stats(ctypes.byref(on), fake, fake, float("nan"), None, None, fake,
+                                 4096, None) == 1
+    assert lib.moe_routing_stats(ctypes.byref(on), fake, fake, 0.01, None, None, fake, 12345,
+                                 None) == 3                              # misaligned workspace
+    bad = native.make_config(8, 128, 4, 2, 128)
+    bad.stats = 2
+    assert native.moe_workspace_bytes(bad) == 0
+    # the statistics scratch is only laid out when asked for
+    big = dict(T=4096, d=4096, E=64, k=2, d_ff=1024)
+    assert (native.moe_workspace_bytes(native.make_config(**big, stats=True))
+            > native.moe_workspace_bytes(native.make_config(**big)))
+    assert ctypes.sizeof(native.MoeRoutingSummary) == 32
