@@ -224,6 +224,88 @@ def dispatch(ids, E: int, C: int | None):
                 row_token=row_token, offsets=offsets)
 
 
+OVERFLOW_DROP = "drop"
+OVERFLOW_REROUTE = "reroute"
+
+
+def dispatch_padded(ids, z, E: int, C: int, overflow: str = OVERFLOW_DROP):
+    """The padded dispatch buffer [E, C, d] and its overflow policy.
+
+    [MoE-S19] "Capacity" / "Visual support": capacity is a tensor dimension; expert e
+    owns slots e*C .. e*C + C - 1, filled in arrival order, empty slots stay padding
+    (the worked case: 16 assignments, 20 slots, 15 filled, 1 dropped).
+    [MoE-S19] "Overflow policies": drop (the route is lost) or reroute (the overflowing
+    route is handled by the next-best expert by score, the router decision overridden).
+
+    Readings (the pages give no algorithm for reroute):
+      * Phase 1 is the drop policy's arrival-order pass, unchanged.
+      * Phase 2 takes the overflowed routes in arrival order (t, then j).  Each goes to
+        the expert ranked best by the token's logits (descending, ties to the lower
+        index) among those the token does not already hold and that still have a free
+        slot; its slot is the next free one.  If there is none it is dropped.
+      * A token's gates are then the gate mode applied to its final experts (slot j's
+        reroute target, or its original expert, dropped or not); tokens without a
+        rerouted route keep their gates.  ``reroute_gates`` does that step.
+
+    Returns a dict:
+      demand[E]       routes asking for each expert before capacity (router's choice)
+      counts[E]       filled slots per expert after the policy
+      final_ids[T,k]  expert that handles each route (the original when not rerouted)
+      rerouted[T,k]   True where phase 2 moved the route
+      route_row[T,k]  e*C + slot of the route, -1 if dropped
+      row_token[E*C]  token in each slot, -1 for padding
+    """
+    ids = np.asarray(ids)
+    T, k = ids.shape
+    if overflow not in (OVERFLOW_DROP, OVERFLOW_REROUTE):
+        raise ValueError(f"unknown overflow policy {overflow!r}")
+    count = np.zeros(E, dtype=np.int64)
+    demand = np.zeros(E, dtype=np.int64)
+    slot = np.full((T, k), -1, dtype=np.int64)
+    final = ids.astype(np.int64).copy()
+    rerouted = np.zeros((T, k), dtype=bool)
+    overflowed = []
+    for t in range(T):                      # phase 1: arrival order
+        for j in range(k):
+            e = int(ids[t, j])
+            if not 0 <= e < E:
+                raise ValueError(f"expert id {e} out of range")
+            demand[e] += 1
+            if count[e] < C:
+                slot[t, j] = count[e]
+                count[e] += 1
+            else:
+                overflowed.append((t, j))
+    if overflow == OVERFLOW_REROUTE:        # phase 2: overflowed routes, arrival order
+        zz = np.asarray(z, dtype=np.float64)
+        for t, j in overflowed:
+            held = set(int(e) for e in final[t])
+            order = sorted(range(E), key=lambda e: (-zz[t, e], e))
+            for e in order:
+                if e not in held and count[e] < C:
+                    final[t, j] = e
+                    slot[t, j] = count[e]
+                    count[e] += 1
+                    rerouted[t, j] = True
+                    break
+    route_row = np.where(slot >= 0, final * C + slot, -1)
+    row_token = np.full(E * C, -1, dtype=np.int64)
+    for t in range(T):
+        for j in range(k):
+            if route_row[t, j] >= 0:
+                row_token[route_row[t, j]] = t
+    return dict(demand=demand, counts=count, final_ids=final, rerouted=rerouted,
+                route_row=route_row, row_token=row_token)
+
+
+def reroute_gates(z, final_ids, g, rerouted, mode: str) -> np.ndarray:
+    """Gates after rerouting: the gate mode over each rerouted token's final experts."""
+    g = np.array(g, dtype=np.float64, copy=True)
+    for t in np.where(np.asarray(rerouted).any(axis=1))[0]:
+        g[t] = gates(np.asarray(z)[t:t + 1], np.asarray(final_ids)[t:t + 1], mode)[0]
+    return g
+
+
 # ----------------------------------------------------------------------------------
 # Compute: SwiGLU expert
 # ----------------------------------------------------------------------------------
@@ -253,7 +335,8 @@ def swiglu_expert(X, w_gate, w_up, w_down) -> np.ndarray:
 # ----------------------------------------------------------------------------------
 
 def moe_layer(x, p: dict, k: int, mode: str, C: int | None = None,
-              add_residual: bool = False, tokens=None, routing=None):
+              add_residual: bool = False, tokens=None, routing=None,
+              layout: str = "ragged", overflow: str = OVERFLOW_DROP):
     """One MoE layer forward, the per-token loop of the pages.
 
     Steps ([MoE-271K] section 3 data path; [MoE-VIS] "Expert Execution"):
@@ -267,8 +350,10 @@ def moe_layer(x, p: dict, k: int, mode: str, C: int | None = None,
 
     ``p`` holds w_router [E,d], logit_bias [E] or None, w_gate/w_up [E,F,d],
     w_down [E,d,F] and optional shared_gate/shared_up [F,d], shared_down [d,F].
-    ``routing`` = (ids, gates) overrides step 1 (used to run the later steps on a
-    given routing).  Returns (y [len(tokens), d], info dict).
+    ``routing`` = (ids, gates) or (ids, gates, logits) overrides step 1 (used to run
+    the later steps on a given routing; the reroute policy needs the logits).
+    ``layout`` "padded" uses the [E, C, d] buffer of ``dispatch_padded`` (C required),
+    with ``overflow`` "drop" or "reroute".  Returns (y [len(tokens), d], info dict).
     """
     x64 = as_f64(x)
     T, d = x64.shape
@@ -277,8 +362,21 @@ def moe_layer(x, p: dict, k: int, mode: str, C: int | None = None,
         ids, g, z = route(x64, p["w_router"], p.get("logit_bias"), k, mode)
     else:
         ids, g = np.asarray(routing[0]), as_f64(routing[1])
-        z = None
-    disp = dispatch(ids, E, C)
+        z = as_f64(routing[2]) if len(routing) > 2 else None
+    if layout == "padded":
+        if C is None:
+            raise ValueError("the padded layout needs a capacity")
+        disp = dispatch_padded(ids, z, E, C, overflow)
+        g = reroute_gates(z, disp["final_ids"], g, disp["rerouted"], mode)
+        disp["offsets"] = np.array([e * C for e in range(E)] + [E * C], dtype=np.int64)
+        seg = [(e * C, e * C + int(disp["counts"][e])) for e in range(E)]
+    elif layout == "ragged":
+        if overflow != OVERFLOW_DROP:
+            raise ValueError("the reroute policy uses the padded layout")
+        disp = dispatch(ids, E, C)
+        seg = [(int(disp["offsets"][e]), int(disp["offsets"][e + 1])) for e in range(E)]
+    else:
+        raise ValueError(f"unknown layout {layout!r}")
     route_row = disp["route_row"]
     tokens = np.arange(T) if tokens is None else np.asarray(tokens)
     want = np.zeros(T, dtype=bool)
@@ -287,7 +385,7 @@ def moe_layer(x, p: dict, k: int, mode: str, C: int | None = None,
     # 3. per expert: gather its kept rows (in packed order) that belong to wanted tokens
     out_rows = {}
     for e in range(E):
-        lo, hi = int(disp["offsets"][e]), int(disp["offsets"][e + 1])
+        lo, hi = seg[e]
         rows = [r for r in range(lo, hi) if want[disp["row_token"][r]]]
         if not rows:
             continue
@@ -368,7 +466,7 @@ def drop_count(demand, C: int | None) -> int:
 
 
 def routing_stats(x, w_router, logit_bias, k: int, C: int | None, alpha: float = 1e-2,
-                  ids=None):
+                  ids=None, overflow: str = OVERFLOW_DROP):
     """Routing statistics of one layer call, in float64.
 
     f_e   fraction of routes dispatched to expert e before capacity (demand_e / (T k));
@@ -381,17 +479,23 @@ def routing_stats(x, w_router, logit_bias, k: int, C: int | None, alpha: float =
     drop  dropped routes / (T k); padding: empty slots / (E C) of the capacity buffer
           ([MoE-S19] Worked case: 20 slots, 15 used, 25% padding); 0 when dropless or
           C = 0 (no slots).
+    With ``overflow`` "reroute" (padded buffer, ``dispatch_padded``) kept counts the
+    routes placed after rerouting; f stays the router's pre-capacity choice.
     Returns a dict with those entries and kept (the number of kept routes).
     """
     z = router_logits(x, w_router, logit_bias)
     T, E = z.shape
     if ids is None:
         ids = top_k(z, k)
-    d = dispatch(ids, E, C)
+    if overflow == OVERFLOW_REROUTE and C is not None:
+        d = dispatch_padded(ids, z, E, C, overflow)
+        kept = int(d["counts"].sum())
+    else:
+        d = dispatch(ids, E, C)
+        kept = int(d["kept"].sum())
     demand = d["demand"].astype(np.float64)
     f = demand / (T * k)
     P = softmax(z).mean(axis=0)
-    kept = int(d["kept"].sum())
     return dict(f=f, P=P, aux=alpha * E * float(np.sum(f * P)), imbalance=imbalance(demand),
                 drop_rate=(T * k - kept) / (T * k),
                 padding_rate=(0.0 if not C else (E * C - kept) / (E * C)), kept=kept)

@@ -440,3 +440,138 @@ def test_routing_stats_drop_and_padding_brute_force():
         P = sum(np.exp(z[t] - z[t].max()) / np.exp(z[t] - z[t].max()).sum() for t in range(T)) / T
         assert np.allclose(st["P"], P, rtol=1e-13, atol=0)
         assert abs(st["aux"] - 1e-2 * E * sum(st["f"][e] * P[e] for e in range(E))) < 1e-15
+
+
+# ---------------------------------------------------------------- padded buffer, reroute
+
+def _worked_logits(g, soft):
+    """Logits consistent with the worked case's assignments: each token's two experts
+    get t1's top-2 logits; t6 (index 5) shares t1's logits, E4 absent from the
+    three-expert reduction (logit -inf)."""
+    z = np.full((g["T"], g["E"]), -np.inf)
+    for t, (a, b) in enumerate(g["assignments"]):
+        z[t, a], z[t, b] = soft["logits"][0], soft["logits"][1]
+    z[5, :3] = soft["logits"]
+    return z
+
+
+def test_padded_buffer_worked_case(golden):
+    """[S19] Visual support - Capacity: the [E, C, d] buffer row by row, 15 of 20 filled."""
+    g = golden("capacity_worked_case.json")
+    d = O.dispatch_padded(np.array(g["assignments"]), None, g["E"], g["C"])
+    for e, toks in enumerate(g["slot_table"]):
+        row = d["row_token"][e * g["C"]:(e + 1) * g["C"]].tolist()
+        assert row == toks + [-1] * (g["C"] - len(toks))
+    assert d["counts"].tolist() == [len(t) for t in g["slot_table"]]
+    assert int(d["counts"].sum()) == g["filled"] and (d["row_token"] < 0).sum() == 5
+    assert [[t, 0] for t in range(g["T"]) if d["route_row"][t, 0] < 0] == g["dropped_routes"]
+    assert not d["rerouted"].any()
+
+
+def test_reroute_worked_case(golden):
+    """[S19] Overflow policies: with reroute, t6's overflowing E1 route is handled by its
+    third-best expert (E3, which has free slots); nothing is dropped, 16 of 20 slots."""
+    g = golden("capacity_worked_case.json")
+    soft = golden("softmax_worked_example.json")
+    ids = np.array(g["assignments"])
+    z = _worked_logits(g, soft)
+    assert np.array_equal(O.top_k(z, 2), ids)       # the logits reproduce the trace
+    d = O.dispatch_padded(ids, z, g["E"], g["C"], O.OVERFLOW_REROUTE)
+    assert d["rerouted"].sum() == 1 and d["rerouted"][5, 0]
+    assert d["final_ids"][5].tolist() == [2, 1]
+    assert d["route_row"][5, 0] == 2 * g["C"] + 3   # E3's 4th slot (3 were filled)
+    assert d["counts"].tolist() == [5, 4, 4, 3] and (d["route_row"] >= 0).all()
+    # gates of t6 over its final experts {E3, E2}, from the printed probabilities
+    p = soft["softmax_3dp"]
+    g_in = O.gates(z, ids, O.GATE_SOFTMAX_TOPK_RENORM)
+    g1 = O.reroute_gates(z, d["final_ids"], g_in, d["rerouted"], O.GATE_SOFTMAX_TOPK_RENORM)
+    assert np.allclose(g1[5], [p[2] / (p[2] + p[1]), p[1] / (p[2] + p[1])], atol=2e-3)
+    g0 = O.reroute_gates(z, d["final_ids"], g_in, d["rerouted"], O.GATE_SOFTMAX_TOPK)
+    assert np.allclose(g0[5], [p[2], p[1]], atol=5e-4)
+    g2 = O.reroute_gates(z, d["final_ids"], g_in, d["rerouted"], O.GATE_TOPK_SOFTMAX)
+    assert abs(g2[5, 0] - 1 / (1 + math.exp(1.6))) < 1e-15   # softmax of (0.2, 1.8)
+    others = np.arange(g["T"]) != 5
+    assert np.array_equal(g1[others], g_in[others])          # untouched tokens keep gates
+
+
+def test_reroute_fills_the_second_expert():
+    """k = 1, E = 2, C = T/2, every token prefers expert 0: the second half of the tokens
+    is rerouted to expert 1, so slot order equals token order."""
+    T = 10
+    z = np.tile([1.0, 0.0], (T, 1))
+    d = O.dispatch_padded(O.top_k(z, 1), z, 2, T // 2, O.OVERFLOW_REROUTE)
+    assert d["route_row"][:, 0].tolist() == list(range(T))
+    assert d["row_token"].tolist() == list(range(T))
+    assert d["rerouted"][:, 0].tolist() == [False] * 5 + [True] * 5
+    drop = O.dispatch_padded(O.top_k(z, 1), z, 2, T // 2)
+    assert drop["route_row"][:, 0].tolist() == list(range(5)) + [-1] * 5
+
+
+def test_reroute_invariants_brute_force():
+    rng = np.random.default_rng(7)
+    for trial in range(40):
+        T, E, k = int(rng.integers(1, 40)), int(rng.integers(2, 8)), 0
+        k = int(rng.integers(1, E + 1))
+        z = np.round(rng.normal(size=(T, E)), 1)
+        ids = O.top_k(z, k)
+        C = int(rng.integers(0, max(1, T * k // E) + 2))
+        drop = O.dispatch_padded(ids, z, E, C)
+        rr = O.dispatch_padded(ids, z, E, C, O.OVERFLOW_REROUTE)
+        ragged = O.dispatch(ids, E, C)
+        # phase 1 equals the drop policy, which equals the ragged dispatch's kept set
+        assert np.array_equal(drop["route_row"] >= 0, ragged["route_row"] >= 0)
+        assert np.array_equal(rr["route_row"][drop["route_row"] >= 0],
+                              drop["route_row"][drop["route_row"] >= 0])
+        assert (rr["counts"] <= C).all() and int(rr["counts"].sum()) == int((rr["route_row"] >= 0).sum())
+        for t in range(T):
+            assert len(set(rr["final_ids"][t].tolist())) == k      # experts stay distinct
+            held = set(rr["final_ids"][t].tolist())
+            rank = sorted(range(E), key=lambda e: (-z[t, e], e))
+            for j in range(k):
+                if rr["route_row"][t, j] < 0:   # dropped: every expert it could take is full
+                    assert all(rr["counts"][e] == C for e in range(E) if e not in held)
+                if rr["rerouted"][t, j]:        # better-ranked candidates are full
+                    tgt = int(rr["final_ids"][t, j])
+                    for e in rank[:rank.index(tgt)]:
+                        assert e in held or rr["counts"][e] == C
+        for r, t in enumerate(rr["row_token"]):
+            if t >= 0:
+                e, s = divmod(r, C)
+                assert s < rr["counts"][e] and t in np.where(rr["route_row"] == r)[0]
+        # capacity large enough: no overflow, both policies equal the dropless order
+        big = O.dispatch_padded(ids, z, E, T * k, O.OVERFLOW_REROUTE)
+        full = O.dispatch(ids, E, None)
+        assert not big["rerouted"].any()
+        for e in range(E):
+            toks = full["row_token"][full["offsets"][e]:full["offsets"][e + 1]].tolist()
+            assert big["row_token"][e * T * k:e * T * k + len(toks)].tolist() == toks
+
+
+def test_padded_layer_equals_ragged_layer():
+    """The buffer layout changes no output; with room for every route, rerouting changes
+    nothing either (dropless)."""
+    rng = np.random.default_rng(11)
+    T, d, E, k, F = 24, 8, 4, 2, 6
+    p = {"w_router": rng.normal(size=(E, d)), "logit_bias": None,
+         "w_gate": rng.normal(size=(E, F, d)), "w_up": rng.normal(size=(E, F, d)),
+         "w_down": rng.normal(size=(E, d, F))}
+    x = rng.normal(size=(T, d))
+    for C in (3, 7, 12):
+        y_r, _ = O.moe_layer(x, p, k, O.GATE_SOFTMAX_TOPK_RENORM, C)
+        y_p, info = O.moe_layer(x, p, k, O.GATE_SOFTMAX_TOPK_RENORM, C, layout="padded")
+        assert np.array_equal(y_r, y_p)
+    y_free, _ = O.moe_layer(x, p, k, O.GATE_TOPK_SOFTMAX, None)
+    y_rr, info = O.moe_layer(x, p, k, O.GATE_TOPK_SOFTMAX, T * k, layout="padded",
+                             overflow=O.OVERFLOW_REROUTE)
+    assert np.array_equal(y_free, y_rr) and not info["rerouted"].any()
+    # tight capacity: rerouted tokens mix their final experts with recomputed gates
+    for C in range(6, 16):
+        y_t, info = O.moe_layer(x, p, k, O.GATE_SOFTMAX_TOPK, C, layout="padded",
+                                overflow=O.OVERFLOW_REROUTE)
+        if info["rerouted"].any():
+            break
+    t = int(np.where(info["rerouted"].any(axis=1))[0][0])
+    sm = O.softmax(O.router_logits(x, p["w_router"])[t])
+    want = sum(sm[e] * O.swiglu_expert(x[t:t + 1], p["w_gate"][e], p["w_up"][e], p["w_down"][e])[0]
+               for j, e in enumerate(info["final_ids"][t]) if info["route_row"][t, j] >= 0)
+    assert np.allclose(y_t[t], want, rtol=1e-12, atol=1e-12)
