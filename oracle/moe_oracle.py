@@ -121,8 +121,12 @@ def gates(z, ids, mode: str) -> np.ndarray:
         if mode == GATE_SOFTMAX_TOPK:
             g[t] = softmax(z[t])[ids[t]]
         elif mode == GATE_SOFTMAX_TOPK_RENORM:
-            p = softmax(z[t])[ids[t]]
-            g[t] = p / np.sum(p)
+            # p_i / sum_sel p_j with p = softmax over all E.  The full softmax's normaliser
+            # cancels in the ratio, so it is evaluated as exp(z_i - c) / sum_sel exp(z_j - c)
+            # with c the largest selected logit: the same value, finite even when every
+            # selected p underflows (a rerouted token may no longer hold its top expert).
+            e = np.exp(sel - np.max(sel))
+            g[t] = e / np.sum(e)
         elif mode == GATE_TOPK_SOFTMAX:
             g[t] = softmax(sel)
         else:
