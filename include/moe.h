@@ -67,6 +67,21 @@ typedef enum {
   MOE_GATE_TOPK_SOFTMAX = 2         /* g = softmax over the k selected logits only       */
 } moe_gate_mode;
 
+/* Where kept routes' rows go ("Mixture-of-Experts: routing and capacity", Capacity and its
+ * Visual support: the dispatch buffer [E, C, d]).                                      */
+typedef enum {
+  MOE_LAYOUT_RAGGED = 0, /* expert segments packed back to back: R rows in total          */
+  MOE_LAYOUT_PADDED = 1  /* expert e owns rows e*C .. e*C + C - 1 (needs capacity >= 0)    */
+} moe_layout;
+
+/* What happens to a route that finds its expert full ("Mixture-of-Experts: routing and
+ * capacity", Overflow policies).                                                       */
+typedef enum {
+  MOE_OVERFLOW_DROP = 0,    /* the route is lost; the token keeps its other gates as they are */
+  MOE_OVERFLOW_REROUTE = 1  /* the route moves to the token's next-best expert with a free
+                             * slot (MOE_LAYOUT_PADDED only; see moe_dispatch)              */
+} moe_overflow;
+
 typedef struct {
   int32_t T;            /* tokens in this call (>= 1)                                   */
   int32_t d;            /* model width                                                   */
@@ -80,6 +95,8 @@ typedef struct {
   int32_t add_residual; /* 1: y = x + MoE(x)                                              */
   int32_t stats;        /* 1: the router also sums each token's full softmax per token
                          *    tile into the workspace, for moe_routing_stats; 0: off     */
+  int32_t layout;       /* moe_layout                                                    */
+  int32_t overflow;     /* moe_overflow                                                  */
 } moe_config;
 /* Supported shapes (else MOE_ERR_UNSUPPORTED): bf16 needs d % 128 == 0 and
  * d_ff % 128 == 0; fp32 needs d % 4 == 0 and d_ff % 4 == 0.                            */
@@ -89,9 +106,10 @@ typedef struct {
  * capacity", Capacity: ceil(8*2/4 * 1.25) = 5).  Returns -1 on invalid arguments.      */
 int32_t moe_capacity(int32_t T, int32_t k, int32_t E, int32_t phi_num, int32_t phi_den);
 
-/* Upper bound on packed rows R: T*k, or E*C when capacity >= 0 and that is smaller.
- * Buffers of packed rows (x_packed, row_token) need this many rows; H and y_packed need
- * moe_max_rows + T rows when has_shared (the shared expert's rows follow the routed). */
+/* Rows of the packed buffer: T*k, or E*C when capacity >= 0 and that is smaller
+ * (MOE_LAYOUT_RAGGED); E*C (MOE_LAYOUT_PADDED).  Buffers of packed rows (x_packed,
+ * row_token) need this many rows; H and y_packed need moe_max_rows + T rows when
+ * has_shared (the shared expert's rows follow the routed ones).                        */
 int64_t moe_max_rows(const moe_config* cfg);
 
 /* Bytes of workspace that moe_forward needs (it keeps every intermediate there); the
@@ -116,22 +134,37 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router,
  * subsection on capacity; "Mixture-of-Experts: routing and capacity", Worked case).
  *   ids        [T, k] int32 (in; ids outside [0,E) or repeated in a token are dropped and
  *              flagged MOE_ERR_BAD_EXPERT_ID in the status word)
- *   x_packed   [moe_max_rows, d] dtype (out): row offsets[e] + p holds x[t] for the p-th
- *              kept route of expert e (tokens ascending)
+ *   gates      [T, k] fp32 (in/out) with MOE_OVERFLOW_REROUTE, else unused (may be NULL)
+ *   x_packed   [moe_max_rows, d] dtype (out): the p-th kept route of expert e (tokens
+ *              ascending) is row offsets[e] + p, holding x[t]
  *   row_token  [moe_max_rows] int32 (out): token of each packed row
  *   route_row  [T, k] int32 (out): packed row of route (t, j), -1 when dropped
- *   offsets    [E + 2] int32 (out): segment starts; offsets[E] = R (kept routes);
- *              offsets[E+1] = R + T with a shared expert, else R
- *   demand     [E] int32 (out): routes asking for each expert before capacity           */
+ *   offsets    int32 (out), the segment table.  MOE_LAYOUT_RAGGED: [E + 2], segment starts;
+ *              offsets[E] = R (kept routes); offsets[E+1] = R + T with a shared expert,
+ *              else R.  MOE_LAYOUT_PADDED: [2E + 2]: offsets[e] = e*C (e <= E),
+ *              offsets[E+1] = E*C (+ T with a shared expert), offsets[E+2+e] = filled
+ *              slots of expert e.  Rows of x_packed past an expert's filled slots are
+ *              not written.
+ *   demand     [E] int32 (out): routes asking for each expert before capacity
+ * MOE_OVERFLOW_REROUTE ("Overflow policies": the overflowing route is handled by the
+ * next-best expert by score): after the arrival-order pass, the routes that overflowed
+ * are taken in arrival order; each moves to the best-ranked expert (logit descending,
+ * ties to the lower index) that its token does not already hold and that has a free
+ * slot, taking the next free slot; with none it is dropped.  A token with a moved route
+ * gets its gates re-evaluated by the gate mode over its final experts (written to
+ * `gates`); other tokens' gates are untouched.  The ranking reads the logits that
+ * moe_route (or moe_forward) left in `ws` for the same config, so `ids` must come from
+ * that call.  The expert that handles route (t, j) is route_row[t, j] / C.             */
 moe_status moe_dispatch(const moe_config* cfg, const void* x, const int32_t* ids,
-                        void* x_packed, int32_t* row_token, int32_t* route_row,
+                        float* gates, void* x_packed, int32_t* row_token, int32_t* route_row,
                         int32_t* offsets, int32_t* demand, void* ws, moe_stream_t stream);
 
-/* Compute: the SwiGLU expert FFNs as grouped GEMMs over the ragged expert segments
+/* Compute: the SwiGLU expert FFNs as grouped GEMMs over the expert segments
  * ("MoE Inference Visualized", Expert Execution: down(SiLU(gate(x)) * up(x));
  * "271,104 Routes...", section 3: one dense matmul per expert batch).
  *   x          [T, d] (A operand of the shared expert; may be NULL without one)
- *   x_packed   [moe_max_rows, d]       offsets [E + 2] from moe_dispatch (device)
+ *   x_packed   [moe_max_rows, d]       offsets: the segment table of moe_dispatch
+ *              (device; with MOE_LAYOUT_PADDED only the filled slots are computed)
  *   w_gate, w_up [E, F, d]   w_down [E, d, F]
  *   shared_gate, shared_up [F, d], shared_down [d, F]: NULL unless has_shared
  *   h          [moe_max_rows (+T), F] dtype (out, intermediate SiLU(g)*u)
@@ -191,7 +224,7 @@ moe_status moe_debug_bounded_wait(void* ws, int64_t limit_ns, moe_stream_t strea
  * all device memory, runtimes with a memory budget fixed before start-up, or hot paths
  * that must not call an allocator (allocation may synchronise or take a global lock).
  * The pages have no counterpart; it is the pack step of moe_dispatch with the same
- * arguments and outputs, minus `ws`.
+ * arguments and outputs, minus `gates` and `ws`.
  *   Scratch: the per-token-tile expert histogram lives in a fixed 64 KiB array inside the
  *   library (16384 int32 entries, held by every device that loads the library until the
  *   process exits).  Configurations whose histogram, ceil(T / tile) * E entries with the
@@ -210,6 +243,8 @@ moe_status moe_dispatch_noalloc(const moe_config* cfg, const void* x, const int3
                                 void* x_packed, int32_t* row_token, int32_t* route_row,
                                 int32_t* offsets, int32_t* demand, int32_t* status,
                                 moe_stream_t stream);
+/*   (MOE_OVERFLOW_REROUTE needs the router's logits in a workspace: it is rejected here
+ *   with MOE_ERR_UNSUPPORTED; both layouts are supported with MOE_OVERFLOW_DROP.)      */
 
 /* Routing statistics of one layer call, written by moe_routing_stats (device memory). */
 typedef struct {

@@ -12,7 +12,7 @@ using namespace moe;
 
 namespace {
 
-constexpr int32_t kAbiVersion = 2;
+constexpr int32_t kAbiVersion = 3;
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
@@ -26,8 +26,16 @@ moe_status validate(const moe_config* c) {
   if ((c->has_shared != 0 && c->has_shared != 1) || (c->add_residual != 0 && c->add_residual != 1) ||
       (c->stats != 0 && c->stats != 1))
     return MOE_ERR_INVALID;
+  if ((c->layout != MOE_LAYOUT_RAGGED && c->layout != MOE_LAYOUT_PADDED) ||
+      (c->overflow != MOE_OVERFLOW_DROP && c->overflow != MOE_OVERFLOW_REROUTE))
+    return MOE_ERR_INVALID;
+  if (c->layout == MOE_LAYOUT_PADDED && c->capacity < 0) return MOE_ERR_INVALID;  // C sizes it
+  if (c->overflow == MOE_OVERFLOW_REROUTE && c->layout != MOE_LAYOUT_PADDED)
+    return MOE_ERR_UNSUPPORTED;
   if (c->E > 256 || c->k > 32) return MOE_ERR_UNSUPPORTED;
   if (c->T > (1 << 24) || static_cast<int64_t>(c->T) * c->k > (INT_MAX / 2)) return MOE_ERR_UNSUPPORTED;
+  if (c->layout == MOE_LAYOUT_PADDED && static_cast<int64_t>(c->E) * c->capacity > (INT_MAX / 2))
+    return MOE_ERR_UNSUPPORTED;
   if (c->dtype == MOE_BF16) {
     if (c->d % 128 != 0 || c->d_ff % 128 != 0) return MOE_ERR_UNSUPPORTED;
   } else {
@@ -37,13 +45,21 @@ moe_status validate(const moe_config* c) {
 }
 
 int64_t max_rows(const moe_config& c) {
+  if (c.layout == MOE_LAYOUT_PADDED)
+    return std::max<int64_t>(static_cast<int64_t>(c.E) * c.capacity, 1);
   int64_t r = static_cast<int64_t>(c.T) * c.k;
   if (c.capacity >= 0) r = std::min<int64_t>(r, static_cast<int64_t>(c.E) * c.capacity);
   return std::max<int64_t>(r, 1);
 }
 
+bool padded(const moe_config& c) { return c.layout == MOE_LAYOUT_PADDED; }
+bool reroute(const moe_config& c) { return c.overflow == MOE_OVERFLOW_REROUTE; }
+// Entries of the segment table (offsets): starts, plus the filled-slot counts when padded.
+size_t offsets_len(const moe_config& c) { return c.E + 2 + (padded(c) ? c.E : 0); }
+
 struct Layout {
-  size_t tile_hist, tile_psum, stats_partial, ids, gates, route_row, row_token, offsets, demand;
+  size_t tile_hist, tile_psum, stats_partial, zkeys, rlist;
+  size_t ids, gates, route_row, row_token, offsets, demand;
   size_t x_packed, h, y_packed;
   size_t scratch_end, total;
   int64_t rmax, rows_h;
@@ -65,12 +81,15 @@ Layout layout_of(const moe_config& c) {
   // Routing statistics (only with cfg.stats): per-tile probability sums and fp64 partials.
   L.tile_psum = c.stats ? take(static_cast<size_t>(num_tiles_for(c.T, c.E)) * c.E * 4) : 0;
   L.stats_partial = c.stats ? take(static_cast<size_t>(kStatsMaxBlocks) * c.E * 8) : 0;
+  // Reroute policy (only with it): the router's ranking keys and the list of moved routes.
+  L.zkeys = reroute(c) ? take(static_cast<size_t>(c.T) * c.E * 4) : 0;
+  L.rlist = reroute(c) ? take((2 * static_cast<size_t>(c.E) * c.capacity + 1) * 4) : 0;
   L.scratch_end = off;
   L.ids = take(Tk * 4);
   L.gates = take(Tk * 4);
   L.route_row = take(Tk * 4);
   L.row_token = take(static_cast<size_t>(L.rmax) * 4);
-  L.offsets = take(static_cast<size_t>(c.E + 2) * 4);
+  L.offsets = take(offsets_len(c) * 4);
   L.demand = take(static_cast<size_t>(c.E) * 4);
   L.x_packed = take(static_cast<size_t>(L.rmax) * c.d * esz);
   L.h = take(static_cast<size_t>(L.rows_h) * c.d_ff * esz);
@@ -121,7 +140,8 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
   const Layout L = layout_of(c);
   int32_t* status = static_cast<int32_t*>(ws);
   int32_t* hist = reinterpret_cast<int32_t*>(at(ws, L.tile_hist));
-  float* psum = c.stats ? reinterpret_cast<float*>(at(ws, L.tile_psum)) : nullptr;
+  const RouterExtras extra{c.stats ? reinterpret_cast<float*>(at(ws, L.tile_psum)) : nullptr,
+                           reroute(c) ? reinterpret_cast<float*>(at(ws, L.zkeys)) : nullptr};
   int32_t* ids = ids_out ? ids_out : reinterpret_cast<int32_t*>(at(ws, L.ids));
   float* gates = gates_out ? gates_out : reinterpret_cast<float*>(at(ws, L.gates));
   int32_t* demand = demand_out ? demand_out : reinterpret_cast<int32_t*>(at(ws, L.demand));
@@ -134,13 +154,18 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
 
   MOE_TRY(record(ev, 0, stream));
   MOE_TRY(cuda_status(
-      launch_router(c, x, w_router, logit_bias, ids, gates, hist, psum, status, stream)));
+      launch_router(c, x, w_router, logit_bias, ids, gates, hist, extra, status, stream)));
   MOE_TRY(record(ev, 1, stream));
   MOE_TRY(cuda_status(launch_dispatch_scatter(c, x, ids, hist, x_packed, row_token, route_row,
                                               offsets, demand, status, stream)));
+  if (reroute(c))
+    MOE_TRY(cuda_status(launch_reroute(c, x, ids, extra.zkeys, gates, x_packed, row_token,
+                                       route_row, offsets,
+                                       reinterpret_cast<int32_t*>(at(ws, L.rlist)), status,
+                                       stream)));
   MOE_TRY(record(ev, 2, stream));
   FfnArgs f{x, x_packed, offsets, w_gate, w_up, w_down, shared_gate, shared_up, shared_down,
-            h, y_packed, L.rmax, status};
+            h, y_packed, L.rmax, status, padded(c) ? offsets + c.E + 2 : nullptr};
   MOE_TRY(ffn(c, f, stream, ev ? static_cast<cudaEvent_t>(ev[3]) : nullptr));
   MOE_TRY(record(ev, 4, stream));
   MOE_TRY(cuda_status(launch_combine(c, y_packed, route_row, gates, offsets, x, y, stream)));
@@ -196,25 +221,31 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router,
   MOE_TRY(check_ws(ws));
   if (!x || !w_router || !ids || !gates) return MOE_ERR_INVALID;
   const Layout L = layout_of(*cfg);
-  return cuda_status(launch_router(
-      *cfg, x, w_router, logit_bias, ids, gates, reinterpret_cast<int32_t*>(at(ws, L.tile_hist)),
-      cfg->stats ? reinterpret_cast<float*>(at(ws, L.tile_psum)) : nullptr,
-      static_cast<int32_t*>(ws), stream));
+  const RouterExtras extra{cfg->stats ? reinterpret_cast<float*>(at(ws, L.tile_psum)) : nullptr,
+                           reroute(*cfg) ? reinterpret_cast<float*>(at(ws, L.zkeys)) : nullptr};
+  return cuda_status(launch_router(*cfg, x, w_router, logit_bias, ids, gates,
+                                   reinterpret_cast<int32_t*>(at(ws, L.tile_hist)), extra,
+                                   static_cast<int32_t*>(ws), stream));
 }
 
 moe_status moe_dispatch(const moe_config* cfg, const void* x, const int32_t* ids,
-                        void* x_packed, int32_t* row_token, int32_t* route_row,
+                        float* gates, void* x_packed, int32_t* row_token, int32_t* route_row,
                         int32_t* offsets, int32_t* demand, void* ws, moe_stream_t stream) {
   MOE_TRY(validate(cfg));
   MOE_TRY(check_ws(ws));
   if (!x || !ids || !x_packed || !row_token || !route_row || !offsets || !demand)
     return MOE_ERR_INVALID;
+  if (reroute(*cfg) && !gates) return MOE_ERR_INVALID;
   const Layout L = layout_of(*cfg);
   int32_t* hist = reinterpret_cast<int32_t*>(at(ws, L.tile_hist));
   int32_t* status = static_cast<int32_t*>(ws);
   MOE_TRY(cuda_status(launch_dispatch_hist(*cfg, ids, hist, status, stream)));
-  return cuda_status(launch_dispatch_scatter(*cfg, x, ids, hist, x_packed, row_token, route_row,
-                                             offsets, demand, status, stream));
+  MOE_TRY(cuda_status(launch_dispatch_scatter(*cfg, x, ids, hist, x_packed, row_token, route_row,
+                                              offsets, demand, status, stream)));
+  if (!reroute(*cfg)) return MOE_OK;
+  return cuda_status(launch_reroute(*cfg, x, ids, reinterpret_cast<const float*>(at(ws, L.zkeys)),
+                                    gates, x_packed, row_token, route_row, offsets,
+                                    reinterpret_cast<int32_t*>(at(ws, L.rlist)), status, stream));
 }
 
 moe_status moe_expert_ffn(const moe_config* cfg, const void* x, const void* x_packed,
@@ -228,7 +259,8 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x, const void* x_pa
     return MOE_ERR_INVALID;
   if (cfg->has_shared && (!x || !shared_gate || !shared_up || !shared_down)) return MOE_ERR_INVALID;
   FfnArgs f{x, x_packed, offsets, w_gate, w_up, w_down, shared_gate, shared_up, shared_down,
-            h, y_packed, max_rows(*cfg), static_cast<int32_t*>(ws)};
+            h, y_packed, max_rows(*cfg), static_cast<int32_t*>(ws),
+            padded(*cfg) ? offsets + cfg->E + 2 : nullptr};
   return ffn(*cfg, f, stream);
 }
 

@@ -17,6 +17,15 @@ constexpr size_t kWsHeaderBytes = 256;
 // Byte offset, in the header, of the ticket counter of the routing-statistics kernel.
 constexpr size_t kWsStatsCounterOffset = 64;
 
+// A route (t, j) is valid if its expert id is in range and not repeated earlier in the
+// token's row of ids.
+__device__ __forceinline__ bool route_id_valid(const int32_t* ids_row, int j, int e, int E) {
+  if (e < 0 || e >= E) return false;
+  for (int q = 0; q < j; ++q)
+    if (ids_row[q] == e) return false;
+  return true;
+}
+
 // First error wins; later errors do not overwrite it.
 __device__ __forceinline__ void record_status(int32_t* status, int32_t code) {
   if (status != nullptr) atomicCAS(status, 0, code);

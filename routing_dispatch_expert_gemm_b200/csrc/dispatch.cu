@@ -24,14 +24,6 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// A route is valid if its expert id is in range and not repeated earlier in the token.
-__device__ __forceinline__ bool route_valid(const int32_t* ids_row, int j, int e, int E) {
-  if (e < 0 || e >= E) return false;
-  for (int q = 0; q < j; ++q)
-    if (ids_row[q] == e) return false;
-  return true;
-}
-
 __global__ void __launch_bounds__(kThreads)
     hist_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int tok_tile,
                 int32_t* __restrict__ tile_hist, int32_t* status) {
@@ -47,7 +39,7 @@ __global__ void __launch_bounds__(kThreads)
     const int t = tok0 + r / k, j = r % k;
     const int32_t* row = ids + static_cast<size_t>(t) * k;
     const int e = row[j];
-    if (route_valid(row, j, e, E))
+    if (route_id_valid(row, j, e, E))
       atomicAdd(&s_hist[e], 1);
     else
       record_status(status, MOE_ERR_BAD_EXPERT_ID);
@@ -61,7 +53,7 @@ struct ScatterArgs {
   const void* x;
   const int32_t* ids;
   const int32_t* tile_hist;
-  int T, d, k, E, tok_tile, num_tiles, capacity, has_shared, copy_round;
+  int T, d, k, E, tok_tile, num_tiles, capacity, has_shared, copy_round, padded;
   void* x_packed;
   int32_t* row_token;
   int32_t* route_row;
@@ -129,12 +121,15 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
     const int tl = r / k, j = r % k;
     const int32_t* row = a.ids + static_cast<size_t>(tile0 + tl) * k;
     const int e = row[j];
-    if (route_valid(row, j, e, E)) atomicOr(&s_mask[e * kWords + (tl >> 5)], 1u << (tl & 31));
+    if (route_id_valid(row, j, e, E)) atomicOr(&s_mask[e * kWords + (tl >> 5)], 1u << (tl & 31));
   }
   __syncthreads();
 
-  // 3. kept counts -> exclusive scan -> offsets (warp 0, 32 experts per step)
-  if (warp == 0) {
+  // 3. kept counts -> exclusive scan -> offsets (warp 0, 32 experts per step); the padded
+  //    buffer gives expert e the fixed rows e*C ..
+  if (a.padded) {
+    for (int e = tid; e <= E; e += kThreads) s_off[e] = e * a.capacity;
+  } else if (warp == 0) {
     int carry = 0;
     for (int base = 0; base < E; base += 32) {
       const int e = base + lane;
@@ -156,6 +151,17 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
     for (int e = tid; e <= E; e += kThreads) a.offsets[e] = s_off[e];
     if (tid == 0) a.offsets[E + 1] = s_off[E] + (a.has_shared ? a.T : 0);
     for (int e = tid; e < E; e += kThreads) a.demand[e] = s_tot[e];
+    if (a.padded)  // filled slots
+      for (int e = tid; e < E; e += kThreads) a.offsets[E + 2 + e] = min(s_tot[e], a.capacity);
+  }
+  if (a.padded) {  // padding slots of the buffer: row_token = -1 (the CTAs share the sweep)
+    const long long slots = static_cast<long long>(E) * a.capacity;
+    for (long long i = static_cast<long long>(blockIdx.x) * kThreads + tid; i < slots;
+         i += static_cast<long long>(gridDim.x) * kThreads) {
+      const int e = static_cast<int>(i / a.capacity);
+      const int p = static_cast<int>(i - static_cast<long long>(e) * a.capacity);
+      if (p >= s_tot[e]) a.row_token[i] = -1;
+    }
   }
 
   // 4. rows of this CTA's tokens' routes
@@ -165,7 +171,7 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
     const int32_t* row = a.ids + static_cast<size_t>(t) * k;
     const int e = row[j];
     int out = -1;
-    if (route_valid(row, j, e, E)) {
+    if (route_id_valid(row, j, e, E)) {
       const uint32_t* m = s_mask + e * kWords;
       int rank = __popc(m[tl >> 5] & ((1u << (tl & 31)) - 1u));
       for (int w = 0; w < (tl >> 5); ++w) rank += __popc(m[w]);
@@ -242,8 +248,8 @@ cudaError_t launch_dispatch_scatter(const moe_config& c, const void* x, const in
   int round = static_cast<int>(kStageBudget / row_bytes);
   round = round < 1 ? 1 : (round > kSubTok ? kSubTok : round);
   ScatterArgs a{x, ids, tile_hist, c.T, c.d, c.k, c.E, kHistTile, num_tiles_for(c.T, c.E),
-                c.capacity, c.has_shared, round, x_packed, row_token, route_row, offsets, demand,
-                status};
+                c.capacity, c.has_shared, round, c.layout == MOE_LAYOUT_PADDED ? 1 : 0, x_packed,
+                row_token, route_row, offsets, demand, status};
   const size_t smem = static_cast<size_t>(round) * row_bytes;
   static bool configured = false;
   if (!configured) {

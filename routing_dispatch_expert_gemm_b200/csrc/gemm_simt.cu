@@ -18,7 +18,8 @@ constexpr int BM = 32, BN = 32, BK = 32, kThreads = 256;
 struct SimtArgs {
   const float* a_routed;   // [Rmax, K]   packed rows (mode gate/up) or H (mode down)
   const float* a_shared;   // [T, K]      x for the shared expert in mode gate/up, else = a_routed
-  const int32_t* offsets;  // [E + 2]
+  const int32_t* offsets;  // [E + 2] segment starts
+  const int32_t* counts;   // [E] routed segment rows (padded layout) or null
   const float* w0;         // [E, N, K]   gate (mode 0) or down (mode 1)
   const float* w1;         // [E, N, K]   up (mode 0)
   const float* w0s;        // [N, K]      shared expert
@@ -27,11 +28,15 @@ struct SimtArgs {
   int E, nseg, K, N;
 };
 
+__device__ __forceinline__ int seg_rows(const SimtArgs& a, int s) {
+  return (a.counts != nullptr && s < a.E) ? a.counts[s] : a.offsets[s + 1] - a.offsets[s];
+}
+
 // Map a linear m-tile index to (segment, m-tile within segment); -1 when past the end.
-__device__ int find_segment(const int32_t* off, int nseg, int mt, int* m_local) {
+__device__ int find_segment(const SimtArgs& a, int nseg, int mt, int* m_local) {
   int acc = 0;
   for (int s = 0; s < nseg; ++s) {
-    const int rows = off[s + 1] - off[s];
+    const int rows = seg_rows(a, s);
     const int n = (rows + BM - 1) / BM;
     if (mt < acc + n) { *m_local = mt - acc; return s; }
     acc += n;
@@ -50,12 +55,12 @@ __global__ void __launch_bounds__(kThreads) simt_kernel(SimtArgs a) {
   __shared__ int s_seg, s_m;
   pdl_trigger();
   pdl_wait();
-  if (threadIdx.x == 0) s_seg = find_segment(a.offsets, a.nseg, blockIdx.x, &s_m);
+  if (threadIdx.x == 0) s_seg = find_segment(a, a.nseg, blockIdx.x, &s_m);
   __syncthreads();
   const int seg = s_seg;
   if (seg < 0) return;
   const int row0 = __ldg(a.offsets + seg);
-  const int rows = __ldg(a.offsets + seg + 1) - row0;
+  const int rows = seg_rows(a, seg);
   const int m0 = s_m * BM, n0 = blockIdx.y * BN;
   const bool shared = seg == a.E;
   // A rows: packed segment for routed experts; for the shared expert in mode 0 the
@@ -111,7 +116,7 @@ cudaError_t launch_ffn_simt(const moe_config& c, const FfnArgs& f, cudaStream_t 
   const long long rows_bound = f.rmax + (c.has_shared ? c.T : 0);
   const int mtiles = static_cast<int>((rows_bound + BM - 1) / BM + nseg);
   SimtArgs g{static_cast<const float*>(f.x_packed), static_cast<const float*>(f.x), f.offsets,
-             static_cast<const float*>(f.w_gate), static_cast<const float*>(f.w_up),
+             f.counts, static_cast<const float*>(f.w_gate), static_cast<const float*>(f.w_up),
              static_cast<const float*>(f.s_gate), static_cast<const float*>(f.s_up),
              static_cast<float*>(f.h), c.E, nseg, c.d, c.d_ff};
   dim3 grid1(mtiles, (c.d_ff + BN - 1) / BN);
@@ -119,7 +124,7 @@ cudaError_t launch_ffn_simt(const moe_config& c, const FfnArgs& f, cudaStream_t 
   if (e != cudaSuccess) return e;
   if (mid != nullptr && (e = record_event(mid, s)) != cudaSuccess) return e;
   SimtArgs g2{static_cast<const float*>(f.h), static_cast<const float*>(f.h), f.offsets,
-              static_cast<const float*>(f.w_down), nullptr, static_cast<const float*>(f.s_down),
+              f.counts, static_cast<const float*>(f.w_down), nullptr, static_cast<const float*>(f.s_down),
               nullptr, static_cast<float*>(f.y_packed), c.E, nseg, c.d_ff, c.d};
   dim3 grid2(mtiles, (c.d + BN - 1) / BN);
   return launch_pdl(simt_kernel<1>, grid2, dim3(kThreads), 0, s, g2);

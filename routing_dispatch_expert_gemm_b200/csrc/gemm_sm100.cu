@@ -80,6 +80,7 @@ struct Maps {
 
 struct Params {
   const int32_t* offsets;  // [nseg + 1] segment row starts
+  const int32_t* counts;   // [E] rows of each routed segment, or null: the gap to the next start
   int nseg, E, K, N;       // N: output columns of the whole problem (F or d)
   __nv_bfloat16* out;
   int ldo;
@@ -95,7 +96,7 @@ struct Cfg {
   static constexpr int OUT_COLS = (MODE == 0) ? BN / 2 : BN;
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int SMEM =
-      1024 + STAGES * STAGE_BYTES + kEpiWarps * kEpiStageBytes + 256 + 2 * kMaxSeg * 4;
+      1024 + STAGES * STAGE_BYTES + kEpiWarps * kEpiStageBytes + 256 + 3 * kMaxSeg * 4;
 };
 
 __device__ __forceinline__ int find_seg(const int* pre, int nseg, int tile) {
@@ -137,6 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 196);
   int* s_pre = reinterpret_cast<int*>(ctl + 256);  // tile prefix per segment
   int* s_row0 = s_pre + kMaxSeg;                   // segment row starts
+  int* s_rows = s_row0 + kMaxSeg;                  // segment row counts
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_blocks = p.N / C::OUT_COLS;
@@ -163,11 +165,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {  // segment table: row starts and exclusive prefix of tile counts
     for (int i = lane; i <= p.nseg; i += 32) s_row0[i] = __ldg(p.offsets + i);
     __syncwarp();
+    for (int i = lane; i < p.nseg; i += 32)
+      s_rows[i] = (p.counts != nullptr && i < p.E) ? __ldg(p.counts + i) : s_row0[i + 1] - s_row0[i];
+    __syncwarp();
     int carry = 0;
     for (int b = 0; b < p.nseg; b += 32) {
       const int s = b + lane;
       int t = 0;
-      if (s < p.nseg) t = ((s_row0[s + 1] - s_row0[s] + BM - 1) / BM) * n_blocks;
+      if (s < p.nseg) t = ((s_rows[s] + BM - 1) / BM) * n_blocks;
       int incl = t;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -192,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool wrapped = false, ok = true;
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
       const int s = find_seg(s_pre, p.nseg, tile);
-      const int mt = (s_row0[s + 1] - s_row0[s] + BM - 1) / BM;
+      const int mt = (s_rows[s] + BM - 1) / BM;
       const int local = tile - s_pre[s];
       const int n = local / mt, m = local - n * mt;
       const bool shared = (s == p.E);
@@ -276,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       const int s = find_seg(s_pre, p.nseg, tile);
-      const int rows = s_row0[s + 1] - s_row0[s];
+      const int rows = s_rows[s];
       const int mt = (rows + BM - 1) / BM;
       const int local = tile - s_pre[s];
       const int n = local / mt, m = local - n * mt;
@@ -406,7 +411,7 @@ cudaError_t launch_ffn_sm100(const moe_config& c, const FfnArgs& f, cudaStream_t
   else
     m1.a_shared = m1.a_routed, m1.b0_shared = m1.b0_routed, m1.b1_shared = m1.b1_routed;
   if (!ok) return cudaErrorInvalidValue;
-  Params p1{f.offsets, nseg, c.E, c.d, c.d_ff, static_cast<__nv_bfloat16*>(f.h), c.d_ff,
+  Params p1{f.offsets, f.counts, nseg, c.E, c.d, c.d_ff, static_cast<__nv_bfloat16*>(f.h), c.d_ff,
             f.status, kWaitLimitNs};
   cudaError_t e = launch_gemm<0, 256>(m1, p1, mt_bound * (c.d_ff / 128), s);
   if (e != cudaSuccess) return e;
@@ -424,8 +429,8 @@ cudaError_t launch_ffn_sm100(const moe_config& c, const FfnArgs& f, cudaStream_t
   m2.b1_routed = m2.b0_routed;
   m2.b1_shared = m2.b0_shared;
   if (!ok) return cudaErrorInvalidValue;
-  Params p2{f.offsets, nseg, c.E, c.d_ff, c.d, static_cast<__nv_bfloat16*>(f.y_packed), c.d,
-            f.status, kWaitLimitNs};
+  Params p2{f.offsets, f.counts, nseg, c.E, c.d_ff, c.d, static_cast<__nv_bfloat16*>(f.y_packed),
+            c.d, f.status, kWaitLimitNs};
   if (c.d % 256 == 0) return launch_gemm<1, 256>(m2, p2, mt_bound * (c.d / 256), s);
   return launch_gemm<1, 128>(m2, p2, mt_bound * (c.d / 128), s);
 }

@@ -14,25 +14,42 @@ constexpr int kHistTile = 128;
 inline int tok_tile_for(int /*T*/, int /*E*/) { return kHistTile; }
 inline int num_tiles_for(int T, int /*E*/) { return (T + kHistTile - 1) / kHistTile; }
 
-// tile_psum (may be null): [num_tiles, E] fp32, the sum over each token tile of every
-// token's full softmax, for the routing statistics.
+// Optional router outputs (null: not written).
+struct RouterExtras {
+  float* tile_psum;  // [num_tiles, E] fp32: per token tile, the sum of every token's full
+                     // softmax (routing statistics)
+  float* zkeys;      // [T, E] fp32: the ranking keys (logit + bias, NaN as -inf) that
+                     // top-k compared (the reroute policy ranks with them)
+};
+
 cudaError_t launch_router(const moe_config& c, const void* x, const void* w_router,
                           const float* bias, int32_t* ids, float* gates, int32_t* tile_hist,
-                          float* tile_psum, int32_t* status, cudaStream_t s);
+                          const RouterExtras& extra, int32_t* status, cudaStream_t s);
 
 // bf16 router on tensor cores (route_sm100.cu); the fp32 router runs on CUDA cores.
 cudaError_t launch_router_sm100(const moe_config& c, const void* x, const void* w_router,
                                 const float* bias, int32_t* ids, float* gates,
-                                int32_t* tile_hist, float* tile_psum, int32_t* status,
-                                cudaStream_t s);
+                                int32_t* tile_hist, const RouterExtras& extra,
+                                int32_t* status, cudaStream_t s);
 
 // Routing statistics from the per-tile probability sums and the dispatch counts.
 // partial: [kStatsMaxBlocks, E] fp64 scratch; counter: zero before the call, left zero.
 constexpr int kStatsMaxBlocks = 148;
+// Kept routes: offsets[E] with the ragged layout, the sum of the filled-slot counts
+// offsets[E+2 ..] with the padded one.
 cudaError_t launch_routing_stats(const moe_config& c, const float* tile_psum,
                                  const int32_t* demand, const int32_t* offsets, float alpha,
                                  double* partial, unsigned int* counter, float* f, float* P,
                                  moe_routing_summary* out, cudaStream_t s);
+
+// Reroute overflow policy on the padded buffer, after the arrival-order pack:
+// assigns the overflowed routes (one CTA, arrival order), rewrites route_row, row_token,
+// the filled-slot counts (offsets[E+2+e]) and the gates of tokens with a moved route,
+// then copies the moved routes' token rows.  list: [2 * E * C + 1] int32 scratch.
+cudaError_t launch_reroute(const moe_config& c, const void* x, const int32_t* ids,
+                           const float* zkeys, float* gates, void* x_packed, int32_t* row_token,
+                           int32_t* route_row, int32_t* offsets, int32_t* list,
+                           int32_t* status, cudaStream_t s);
 
 cudaError_t launch_dispatch_hist(const moe_config& c, const int32_t* ids, int32_t* tile_hist,
                                  int32_t* status, cudaStream_t s);
@@ -60,6 +77,8 @@ struct FfnArgs {
   void* y_packed;         // [Rmax (+T), d]
   int64_t rmax;           // rows of x_packed
   int32_t* status;
+  const int32_t* counts;  // [E] rows of each routed segment (padded layout), or null:
+                          // rows = offsets[s + 1] - offsets[s]
 };
 
 // fp32 path: CUDA-core grouped GEMMs.  `mid` (may be null) is recorded between the

@@ -59,7 +59,16 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_config* cfg, const void* x,
   if (cfg == nullptr || cfg->T < 1 || cfg->d < 1 || cfg->E < 1 || cfg->k < 1 || cfg->k > cfg->E ||
       (cfg->dtype != MOE_F32 && cfg->dtype != MOE_BF16))
     return MOE_ERR_INVALID;
+  if ((cfg->layout != MOE_LAYOUT_RAGGED && cfg->layout != MOE_LAYOUT_PADDED) ||
+      (cfg->overflow != MOE_OVERFLOW_DROP && cfg->overflow != MOE_OVERFLOW_REROUTE) ||
+      (cfg->layout == MOE_LAYOUT_PADDED && cfg->capacity < 0))
+    return MOE_ERR_INVALID;
+  // The reroute policy ranks with the router's logits, which live in a workspace.
+  if (cfg->overflow == MOE_OVERFLOW_REROUTE) return MOE_ERR_UNSUPPORTED;
   if (cfg->E > 256 || cfg->k > 32 || cfg->T > (1 << 24)) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(cfg->T) * cfg->k > (1 << 30) ||
+      (cfg->layout == MOE_LAYOUT_PADDED && static_cast<long long>(cfg->E) * cfg->capacity > (1 << 30)))
+    return MOE_ERR_UNSUPPORTED;
   if ((cfg->dtype == MOE_BF16 && cfg->d % 128 != 0) || (cfg->dtype == MOE_F32 && cfg->d % 4 != 0))
     return MOE_ERR_UNSUPPORTED;
   if (!x || !ids || !x_packed || !row_token || !route_row || !offsets || !demand)

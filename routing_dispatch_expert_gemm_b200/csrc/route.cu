@@ -38,6 +38,7 @@ struct RouterArgs {
   float* gates;
   int32_t* tile_hist;
   float* tile_psum;  // null: no routing statistics
+  float* zkeys;      // null: ranking keys not stored
 };
 
 // NaN logits rank as -inf so that k valid experts are always selected.
@@ -159,6 +160,8 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(RouterArgs a) {
         const float z = warp_reduce_experts<EP>(acc[i], lane);
         const int ge = p * EP + (lane % EP);
         const float zb = (ge < a.E && a.bias != nullptr) ? z + __ldg(a.bias + ge) : z;
+        if (a.zkeys != nullptr && tok[i] < tok_end && lane < EP && ge < a.E)
+          a.zkeys[static_cast<size_t>(tok[i]) * a.E + ge] = rank_key(zb);
 #pragma unroll
         for (int q = 0; q < NP; ++q)
           if (q == p) zl[i][q] = zb;
@@ -280,11 +283,11 @@ cudaError_t launch_typed(RouterArgs a, cudaStream_t s) {
 
 cudaError_t launch_router(const moe_config& c, const void* x, const void* w_router,
                           const float* bias, int32_t* ids, float* gates, int32_t* tile_hist,
-                          float* tile_psum, int32_t* status, cudaStream_t s) {
+                          const RouterExtras& extra, int32_t* status, cudaStream_t s) {
   if (c.dtype == MOE_BF16)
-    return launch_router_sm100(c, x, w_router, bias, ids, gates, tile_hist, tile_psum, status, s);
+    return launch_router_sm100(c, x, w_router, bias, ids, gates, tile_hist, extra, status, s);
   RouterArgs a{x, w_router, bias, c.T, c.d, c.E, c.k, c.gate_mode, kHistTile, 0,
-               ids, gates, tile_hist, tile_psum};
+               ids, gates, tile_hist, extra.tile_psum, extra.zkeys};
   return launch_typed<float>(a, s);
 }
 

@@ -52,6 +52,7 @@ struct RouteParams {
   float* gates;
   int32_t* tile_hist;
   float* tile_psum;  // null: no routing statistics
+  float* zkeys;      // null: ranking keys not stored
   int32_t* status;
   int64_t limit_ns;
 };
@@ -249,6 +250,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < EN_T; ++e) zr[e] = (e < p.E) ? rank_key(zr[e] + s_bias[e]) : -INFINITY;
+        if (p.zkeys != nullptr && t < p.T) {
+          float* zrow = p.zkeys + static_cast<size_t>(t) * p.E;
+#pragma unroll
+          for (int e = 0; e < EN_T; ++e)
+            if (e < p.E) zrow[e] = zr[e];
+        }
         topk_tournament<EN_T, KMAX>(zr, p.E, p.k, tv, te);
       } else {
         for (int c0 = 0; c0 < p.EN; c0 += 16) {
@@ -260,6 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int e = c0 + j;
             if (e < p.E) {
               const float v = rank_key(__uint_as_float(r[j]) + s_bias[e]);
+              if (p.zkeys != nullptr && t < p.T) p.zkeys[static_cast<size_t>(t) * p.E + e] = v;
               if (ranks_before(v, e, tv[KMAX - 1], te[KMAX - 1])) {
                 tv[KMAX - 1] = v;
                 te[KMAX - 1] = e;
@@ -385,8 +393,9 @@ cudaError_t launch_en(const RouteMaps& maps, const RouteParams& p, int grid, int
 
 cudaError_t launch_router_sm100(const moe_config& c, const void* x, const void* w_router,
                                 const float* bias, int32_t* ids, float* gates,
-                                int32_t* tile_hist, float* tile_psum, int32_t* status,
-                                cudaStream_t s) {
+                                int32_t* tile_hist, const RouterExtras& extra,
+                                int32_t* status, cudaStream_t s) {
+  float* tile_psum = extra.tile_psum;
   // Logit columns (MMA N): 16, 32 or 64 when E fits, so the epilogue can keep a token's
   // logits in registers; otherwise E rounded up to a multiple of 16.
   const int EN = c.E <= 16 ? 16 : c.E <= 32 ? 32 : c.E <= 64 ? 64 : ((c.E + 15) / 16) * 16;
@@ -402,7 +411,7 @@ cudaError_t launch_router_sm100(const moe_config& c, const void* x, const void* 
       !encode_2d_box(&maps.w, w_router, c.d, c.E, EN))
     return cudaErrorInvalidValue;
   RouteParams p{bias, c.T, c.d, c.E, c.k, EN, c.gate_mode, stages, cols,
-                ids, gates, tile_hist, tile_psum, status, kWaitLimitNs};
+                ids, gates, tile_hist, tile_psum, extra.zkeys, status, kWaitLimitNs};
   const int grid = (c.T + kTokens - 1) / kTokens;
   const int smem = 1024 + stages * stage_bytes + 256 + 2 * 256 * 4 + (tile_psum ? 4 * 256 * 4 : 0);
   if (EN == 16) return launch_en<16>(maps, p, grid, smem, s);

@@ -32,7 +32,7 @@ struct StatsArgs {
   float* f;                 // [E] or null
   float* P;                 // [E] or null
   moe_routing_summary* out;
-  int T, E, k, C, ntiles, chunk;
+  int T, E, k, C, ntiles, chunk, padded;
   float alpha;
 };
 
@@ -92,8 +92,12 @@ __global__ void __launch_bounds__(kThreads) stats_kernel(StatsArgs a) {
     }
     __syncthreads();
   }
-  if (e == 0) {
-    const int R = __ldcg(a.offsets + a.E);
+  if (e == 0) {  // kept routes: the ragged segment end, or the padded buffer's filled slots
+    int R = 0;
+    if (a.padded)
+      for (int q = 0; q < a.E; ++q) R += __ldcg(a.offsets + a.E + 2 + q);
+    else
+      R = __ldcg(a.offsets + a.E);
     const long long Tk = static_cast<long long>(a.T) * a.k;
     const double mean = static_cast<double>(s_sum[0]) / a.E;
     moe_routing_summary r;
@@ -123,7 +127,7 @@ cudaError_t launch_routing_stats(const moe_config& c, const float* tile_psum,
   if (nb < 1) nb = 1;
   const int chunk = (ntiles + nb - 1) / nb;
   StatsArgs a{tile_psum, demand, offsets, partial, counter, f, P, out,
-              c.T, c.E, c.k, c.capacity, ntiles, chunk, alpha};
+              c.T, c.E, c.k, c.capacity, ntiles, chunk, c.layout == MOE_LAYOUT_PADDED ? 1 : 0, alpha};
   return launch_pdl(stats_kernel, dim3(nb), dim3(kThreads), 0, s, a);
 }
 

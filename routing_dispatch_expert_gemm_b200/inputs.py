@@ -140,3 +140,18 @@ def random_ids(T: int, E: int, k: int, seed: int = 0, skew: float = 1.0) -> torc
     w = torch.tensor([(e + 1.0) ** -skew for e in range(E)])
     ids = torch.stack([torch.multinomial(w, k, replacement=False, generator=gen) for _ in range(T)])
     return ids.to(torch.int32)
+
+
+def integer_router(wl: Workload, seed: int = 0, device="cpu", bias=None):
+    """Token states and router weights with small integer values (|x| <= 3, |w| <= 2) and an
+    optional integer logit bias.  Every product and partial sum of the logit contraction is
+    an integer below 2**24, so fp32 accumulation in any order gives the exact logits: the
+    GPU and an fp64 reference then rank experts identically, exact ties included.  Used to
+    test the reroute policy, whose cascade depends on the full ranking of each token.
+    Returns (x [T, d], w_router [E, d], logit_bias [E] fp32 or None)."""
+    gen = torch.Generator(device="cpu").manual_seed(seed)
+    dt = wl.torch_dtype
+    x = torch.randint(-3, 4, (wl.T, wl.d), generator=gen).to(dt).to(device)
+    w = torch.randint(-2, 3, (wl.E, wl.d), generator=gen).to(dt).to(device)
+    b = None if bias is None else torch.tensor([float(v) for v in bias], device=device)
+    return x, w, b

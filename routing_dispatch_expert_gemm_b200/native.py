@@ -13,12 +13,14 @@ import os
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
 
 MOE_OK = 0
-ABI_VERSION = 2  # moe_abi_version() of the library this binding mirrors
+ABI_VERSION = 3  # moe_abi_version() of the library this binding mirrors
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID", 2: "MOE_ERR_UNSUPPORTED",
                 3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_BAD_EXPERT_ID",
                 6: "MOE_ERR_TIMEOUT"}
 DTYPES = {"f32": 0, "bf16": 1}
 GATE_MODES = {"softmax_topk": 0, "softmax_topk_renorm": 1, "topk_softmax": 2}
+LAYOUTS = {"ragged": 0, "padded": 1}
+OVERFLOWS = {"drop": 0, "reroute": 1}
 
 # Every symbol include/moe.h declares (checked by the CPU test suite).
 EXPORTS = ("moe_capacity", "moe_max_rows", "moe_workspace_bytes", "moe_workspace_init",
@@ -37,17 +39,25 @@ class MoeError(RuntimeError):
 class MoeConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("T", "d", "E", "k", "d_ff", "dtype", "gate_mode", "capacity",
-                 "has_shared", "add_residual", "stats")]
+                 "has_shared", "add_residual", "stats", "layout", "overflow")]
 
     def __repr__(self):
         return "MoeConfig(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
 
 
 def make_config(T, d, E, k, d_ff, dtype="bf16", gate_mode="topk_softmax", capacity=-1,
-                has_shared=False, add_residual=False, stats=False) -> MoeConfig:
+                has_shared=False, add_residual=False, stats=False, layout="ragged",
+                overflow="drop") -> MoeConfig:
     return MoeConfig(int(T), int(d), int(E), int(k), int(d_ff), DTYPES[dtype],
                      GATE_MODES[gate_mode], int(capacity), int(bool(has_shared)),
-                     int(bool(add_residual)), int(bool(stats)))
+                     int(bool(add_residual)), int(bool(stats)), LAYOUTS[layout],
+                     OVERFLOWS[overflow])
+
+
+def offsets_len(cfg: MoeConfig) -> int:
+    """Entries of the segment table moe_dispatch writes: E + 2, plus E filled-slot counts
+    with the padded layout."""
+    return cfg.E + 2 + (cfg.E if cfg.layout == LAYOUTS["padded"] else 0)
 
 
 class MoeRoutingSummary(ctypes.Structure):
@@ -85,7 +95,7 @@ def lib() -> ctypes.CDLL:
             "moe_workspace_bytes": (ctypes.c_size_t, [_CFG]),
             "moe_workspace_init": (_I32, [_P, _P]),
             "moe_route": (_I32, [_CFG, _P, _P, _P, _P, _P, _P, _P]),
-            "moe_dispatch": (_I32, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+            "moe_dispatch": (_I32, [_CFG] + [_P] * 10),
             "moe_expert_ffn": (_I32, [_CFG] + [_P] * 12 + [_P]),
             "moe_combine": (_I32, [_CFG, _P, _P, _P, _P, _P, _P, _P]),
             "moe_forward": (_I32, [_CFG] + [_P] * 15 + [_P]),
@@ -160,10 +170,12 @@ def moe_route(cfg, x, w_router, logit_bias, ids, gates, ws, stream=None):
                            _ptr(ids), _ptr(gates), _ptr(ws), _stream(stream)), "moe_route")
 
 
-def moe_dispatch(cfg, x, ids, x_packed, row_token, route_row, offsets, demand, ws, stream=None):
-    _check(lib().moe_dispatch(ctypes.byref(cfg), _ptr(x), _ptr(ids), _ptr(x_packed),
-                              _ptr(row_token), _ptr(route_row), _ptr(offsets), _ptr(demand),
-                              _ptr(ws), _stream(stream)), "moe_dispatch")
+def moe_dispatch(cfg, x, ids, gates, x_packed, row_token, route_row, offsets, demand, ws,
+                 stream=None):
+    """``gates`` is read and rewritten with the reroute policy; otherwise it may be None."""
+    _check(lib().moe_dispatch(ctypes.byref(cfg), _ptr(x), _ptr(ids), _ptr(gates),
+                              _ptr(x_packed), _ptr(row_token), _ptr(route_row), _ptr(offsets),
+                              _ptr(demand), _ptr(ws), _stream(stream)), "moe_dispatch")
 
 
 def moe_expert_ffn(cfg, x, x_packed, offsets, w_gate, w_up, w_down, shared_gate, shared_up,

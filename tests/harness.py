@@ -62,7 +62,7 @@ def staged_gpu(cfg, x, p, ids, gates, ws=None):
     route_row = torch.empty((T, k), dtype=torch.int32, device=dev)
     offsets = torch.empty(E + 2, dtype=torch.int32, device=dev)
     demand = torch.empty(E, dtype=torch.int32, device=dev)
-    N.moe_dispatch(cfg, x, ids, xp, row_token, route_row, offsets, demand, ws)
+    N.moe_dispatch(cfg, x, ids, None, xp, row_token, route_row, offsets, demand, ws)
     h = torch.empty((rows_h, cfg.d_ff), dtype=x.dtype, device=dev)
     yp = torch.empty((rows_h, cfg.d), dtype=x.dtype, device=dev)
     N.moe_expert_ffn(cfg, x, xp, offsets, p["w_gate"], p["w_up"], p["w_down"], p["shared_gate"],

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(native):
     lib = ctypes.CDLL(native.LIB_PATH)
     for name in declared:
         assert hasattr(lib, name), name
-    assert native.moe_abi_version() == native.ABI_VERSION == 2
+    assert native.moe_abi_version() == native.ABI_VERSION == 3
 
 
 def test_library_is_sm100a_build(native):
@@ -92,7 +92,11 @@ def test_errors_return_before_any_launch(native):
     assert lib.moe_route(ctypes.byref(cfg), fake, fake, None, fake, fake, None, None) == 3
     # null required pointers
     assert lib.moe_route(ctypes.byref(cfg), None, fake, None, fake, fake, 4096, None) == 1
-    assert lib.moe_dispatch(ctypes.byref(cfg), fake, None, fake, fake, fake, fake, fake,
+    assert lib.moe_dispatch(ctypes.byref(cfg), fake, None, None, fake, fake, fake, fake, fake,
+                            4096, None) == 1
+    # the reroute policy rewrites the gates: they are required
+    rr = native.make_config(8, 128, 4, 2, 128, capacity=4, layout="padded", overflow="reroute")
+    assert lib.moe_dispatch(ctypes.byref(rr), fake, fake, None, fake, fake, fake, fake, fake,
                             4096, None) == 1
     assert lib.moe_combine(ctypes.byref(cfg), fake, fake, fake, None, None, None, None) == 1
     res = native.make_config(8, 128, 4, 2, 128, add_residual=True)
@@ -128,3 +132,29 @@ def test_routing_stats_arguments(native):
     assert (native.moe_workspace_bytes(native.make_config(**big, stats=True))
             > native.moe_workspace_bytes(native.make_config(**big)))
     assert ctypes.sizeof(native.MoeRoutingSummary) == 32
+
+
+def test_layout_and_overflow_validation(native):
+    # the padded buffer is sized by the capacity; reroute needs the padded buffer
+    assert native.moe_workspace_bytes(native.make_config(8, 128, 4, 2, 128, layout="padded")) == 0
+    assert native.moe_workspace_bytes(native.make_config(
+        8, 128, 4, 2, 128, capacity=4, overflow="reroute")) == 0
+    bad = native.make_config(8, 128, 4, 2, 128, capacity=4)
+    bad.layout = 2
+    assert native.moe_workspace_bytes(bad) == 0
+    pad = native.make_config(1000, 128, 8, 2, 256, capacity=300, layout="padded")
+    assert native.moe_max_rows(pad) == 8 * 300                 # E*C even above T*k
+    rag = native.make_config(1000, 128, 8, 2, 256, capacity=300)
+    assert native.moe_max_rows(rag) == 2000
+    assert native.offsets_len(pad) == 2 * 8 + 2 and native.offsets_len(rag) == 8 + 2
+    rr = native.make_config(1000, 128, 8, 2, 256, capacity=300, layout="padded",
+                            overflow="reroute")
+    assert native.moe_workspace_bytes(rr) > native.moe_workspace_bytes(pad)
+    lib = native.lib()
+    fake = 1 << 20
+    # no workspace for the router's logits: reroute is unsupported without allocation
+    assert lib.moe_dispatch_noalloc(ctypes.byref(rr), fake, fake, fake, fake, fake, fake,
+                                    fake, None, None) == 2
+    assert lib.moe_dispatch_noalloc(ctypes.byref(native.make_config(
+        8, 128, 4, 2, 128, layout="padded")), fake, fake, fake, fake, fake, fake, fake, None,
+        None) == 1

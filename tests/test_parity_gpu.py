@@ -104,7 +104,7 @@ def test_dispatch_bit_exact(T, E, k, skew, cap):
     route_row = torch.empty((T, k), dtype=torch.int32, device="cuda")
     offsets = torch.empty(E + 2, dtype=torch.int32, device="cuda")
     demand = torch.empty(E, dtype=torch.int32, device="cuda")
-    N.moe_dispatch(cfg, xd, idsd, xp, row_token, route_row, offsets, demand, ws)
+    N.moe_dispatch(cfg, xd, idsd, None, xp, row_token, route_row, offsets, demand, ws)
     assert N.moe_get_device_status(ws) == 0
     ref = O.dispatch(ids.numpy(), E, cap)
     R = int(ref["offsets"][E])
@@ -133,7 +133,7 @@ def test_dispatch_rejects_bad_ids():
     route_row = torch.empty((T, k), dtype=torch.int32, device="cuda")
     offsets = torch.empty(E + 2, dtype=torch.int32, device="cuda")
     demand = torch.empty(E, dtype=torch.int32, device="cuda")
-    N.moe_dispatch(cfg, x, ids.cuda(), xp, row_token, route_row, offsets, demand, ws)
+    N.moe_dispatch(cfg, x, ids.cuda(), None, xp, row_token, route_row, offsets, demand, ws)
     assert N.moe_get_device_status(ws, clear=True) == 5      # MOE_ERR_BAD_EXPERT_ID
     assert N.moe_get_device_status(ws) == 0
     rr = route_row.cpu()

@@ -61,7 +61,7 @@ def _route_dispatch_stats(wl, cfg, x, p, ws):
     route_row = torch.empty((T, k), dtype=torch.int32, device=dev)
     offsets = torch.empty(E + 2, dtype=torch.int32, device=dev)
     demand = torch.empty(E, dtype=torch.int32, device=dev)
-    N.moe_dispatch(cfg, x, ids, xp, row_token, route_row, offsets, demand, ws)
+    N.moe_dispatch(cfg, x, ids, None, xp, row_token, route_row, offsets, demand, ws)
     f = torch.full((E,), -1.0, device=dev)
     P = torch.full((E,), -1.0, device=dev)
     summ = torch.zeros(32, dtype=torch.uint8, device=dev)

@@ -44,7 +44,7 @@ def test_noalloc_dispatch_matches_workspace_dispatch_twice():
         x = torch.randn((T, d), generator=torch.Generator().manual_seed(E)).to(torch.bfloat16).to(dev)
         ref = _outputs(cfg, d, dev)
         ws = N.workspace(cfg)
-        N.moe_dispatch(cfg, x, ids, ref["x_packed"], ref["row_token"], ref["route_row"],
+        N.moe_dispatch(cfg, x, ids, None, ref["x_packed"], ref["row_token"], ref["route_row"],
                        ref["offsets"], ref["demand"], ws)
         assert N.moe_get_device_status(ws) == 0
         out = _outputs(cfg, d, dev)
