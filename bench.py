@@ -34,9 +34,11 @@ METRIC = "routed tokens/s per MoE layer fwd (1×B200) + % of bf16 TC / HBM roofl
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNELS = ["route", "pack", "gemm_gate_up", "gemm_down", "combine"]
-KERNEL_SOURCES = {"route": ["route.cu"], "pack": ["dispatch.cu"],
+KERNEL_SOURCES = {"route": ["route.cu", "route_sm100.cu", "common.cuh"],
+                  "pack": ["dispatch.cu", "reroute.cu", "common.cuh"],
                   "gemm_gate_up": ["gemm_sm100.cu", "common.cuh"],
-                  "gemm_down": ["gemm_sm100.cu", "common.cuh"], "combine": ["combine.cu"]}
+                  "gemm_down": ["gemm_sm100.cu", "common.cuh"],
+                  "combine": ["combine.cu", "common.cuh"]}
 
 
 def parse_args():
@@ -215,7 +217,8 @@ def oracle_sample_rate(wl, x, layers, budget_s=12.0, max_layers=None, n_tokens=N
     done = 0
     xin = x
     for p in layers:
-        y, _ = O.moe_layer(xin, p, wl.k, wl.gate_mode, C, add_residual=wl.add_residual, tokens=toks)
+        y, _ = O.moe_layer(xin, p, wl.k, wl.gate_mode, C, add_residual=wl.add_residual, tokens=toks,
+                           layout=wl.layout, overflow=wl.overflow)
         done += 1
         if wl.add_residual and toks is None:
             xin = O.round_to_bf16(y) if wl.dtype == "bf16" else y
@@ -258,11 +261,12 @@ def run_ours(a):
     x, layers = I.make_inputs(wl, seed=a.seed + rank, device=dev)
     cap = -1 if wl.phi is None else N.moe_capacity(wl.T, wl.k, wl.E, *wl.phi)
     cfg = N.make_config(wl.T, wl.d, wl.E, wl.k, wl.d_ff, dtype=wl.dtype, gate_mode=wl.gate_mode,
-                        capacity=cap, has_shared=wl.has_shared, add_residual=wl.add_residual)
+                        capacity=cap, has_shared=wl.has_shared, add_residual=wl.add_residual,
+                        layout=wl.layout, overflow=wl.overflow)
     ws = N.workspace(cfg, dev)
     ybuf = [torch.empty_like(x), torch.empty_like(x)]
     demand = torch.zeros((L, wl.E), dtype=torch.int32, device=dev)
-    offsets = torch.zeros((L, wl.E + 2), dtype=torch.int32, device=dev)
+    offsets = torch.zeros((L, N.offsets_len(cfg)), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step(xin, evs=None):
@@ -381,8 +385,12 @@ def run_ours(a):
 
     dem = demand.cpu()
     offs = offsets.cpu()
-    Rs = [int(offs[l, wl.E]) for l in range(L)]
-    touched = [int((offs[l, 1:wl.E + 1] - offs[l, :wl.E] > 0).sum()) for l in range(L)]
+    if wl.layout == "padded":  # filled slots per expert follow the segment starts
+        Rs = [int(offs[l, wl.E + 2:].sum()) for l in range(L)]
+        touched = [int((offs[l, wl.E + 2:] > 0).sum()) for l in range(L)]
+    else:
+        Rs = [int(offs[l, wl.E]) for l in range(L)]
+        touched = [int((offs[l, 1:wl.E + 1] - offs[l, :wl.E] > 0).sum()) for l in range(L)]
     costs = [kernel_costs(wl, R, tc) for R, tc in zip(Rs, touched)]
     peaks, peak_src = load_peaks()
     # Tensor peak for the clock regime actually seen: the burst figure when the SM clock
@@ -484,12 +492,13 @@ def run_ours(a):
         "config": {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k,
                    "d_ff": wl.d_ff, "layers": L, "gate_mode": wl.gate_mode,
                    "capacity": cap, "shared_expert": wl.has_shared,
-                   "residual": wl.add_residual, "parallelism": f"replicas{world}",
+                   "residual": wl.add_residual, "layout": wl.layout, "overflow": wl.overflow,
+                   "parallelism": f"replicas{world}",
                    "cuda_graph": a.graph,
                    "l2": ("flushed between steps" if flush is not None else
                           f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB of weights per step)")},
         "roofline": roofline, "kernels": breakdown, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": a.steps * L * 5, "clocks": clk,
+        "gpu_launches": a.steps * L * (7 if wl.overflow == "reroute" else 5), "clocks": clk,
         "routes_per_step": int(dem.sum()), "output_finite": bool(ok_out),
     }
     print(json.dumps(out), flush=True)
@@ -530,7 +539,8 @@ def run_reference(a):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k,
-                   "d_ff": wl.d_ff, "layers": wl.layers, "gate_mode": wl.gate_mode},
+                   "d_ff": wl.d_ff, "layers": wl.layers, "gate_mode": wl.gate_mode,
+                   "layout": wl.layout, "overflow": wl.overflow},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": "per step: " + sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -5,15 +5,18 @@
 // route is handled by the next-best expert by score, the router's decision overridden).
 //
 // Runs after the arrival-order pack, which has already placed every route that fit and
-// left route_row = -1 on the ones that overflowed.  The reroute itself is sequential by
+// left route_row = -1 on the ones that overflowed.  The reroute is sequential by
 // definition: whether a route finds a free slot depends on every earlier reroute.  One CTA
-// therefore walks the overflowed routes in arrival order (t, then j): each chunk of 256
-// routes is compacted with a block-wide scan, then warp 0 places the chunk's overflowed
-// routes one at a time.  For each, the 32 lanes take an arg-max over the experts the token
-// does not hold and that still have a free slot, ordered by (ranking key descending, expert
-// index ascending), the router's own order and tie rule on the router's own keys.  The walk
-// stops as soon as no slot is free.  A token with a moved route gets its gates recomputed by
-// the gate mode over its final experts.  A second kernel copies the moved routes' rows.
+// walks the routes in chunks: all threads compact a chunk's overflowed routes (arrival
+// order) and stage their tokens' ranking keys and expert ids in shared memory; then one
+// warp places them one at a time.  In that warp lane l owns experts l, l+32, ..: it keeps
+// their filled-slot counts and the current token's "already held" flags in registers, so a
+// placement is a warp max over an order-preserving integer code of the key (free, not held
+// experts only) and a warp min of the expert index among the maxima -- the router's order
+// and tie rule on the router's own keys -- with no memory round trip on the critical path.
+// The walk stops as soon as no slot is free; the loop keeps all its state in registers and
+// only issues stores.  A second, grid-wide kernel copies each moved route's token row and
+// re-evaluates that token's gates by the gate mode over its final experts.
 #include <climits>
 
 #include "common.cuh"
@@ -22,18 +25,21 @@
 namespace moe {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 256;  // copy kernel
 constexpr int kWarps = kThreads / 32;
+constexpr int kAssignThreads = 512;
+constexpr int kAssignWarps = kAssignThreads / 32;
+constexpr int kStageFloats = 16384;  // staged keys per chunk (64 KB)
+constexpr int kStageIds = 16384;     // staged expert ids per chunk (64 KB)
 
 struct AssignArgs {
   const int32_t* ids;    // [T, k]
   const float* zkeys;    // [T, E]
-  float* gates;          // [T, k]
   int32_t* row_token;    // [E * C]
   int32_t* route_row;    // [T, k]
   int32_t* offsets;      // segment table; filled-slot counts at offsets[E + 2 + e]
   int32_t* list;         // [0]: moved routes n, then n (token, row) pairs
-  int T, k, E, C, gate_mode;
+  int T, k, E, C, chunk;
 };
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -48,14 +54,28 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Gates of token t over its final experts fin[0..k) (warp-wide; lane j < k owns slot j).
-__device__ void regate(const AssignArgs& a, int t, const int* fin, int lane) {
-  const float* zrow = a.zkeys + static_cast<size_t>(t) * a.E;
-  const int e = (lane < a.k) ? fin[lane] : -1;
-  const bool valid = e >= 0 && e < a.E;
+// Order-preserving map of a ranking key (never NaN) to a nonzero unsigned code: a larger
+// key gives a larger code, -0 and +0 the same one, and -inf the smallest (still > 0).
+__device__ __forceinline__ uint32_t key_code(float z) {
+  if (z == 0.f) z = 0.f;
+  const uint32_t u = __float_as_uint(z);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Gates of token t over its final experts (warp-wide; lane j < k writes slot j).  Slot j's
+// expert is the one whose block holds its row, or its original expert when it was dropped.
+__device__ void regate(const int32_t* ids, const float* zkeys, const int32_t* route_row,
+                       float* gates, int t, int k, int E, int C, int gate_mode, int lane) {
+  const float* zrow = zkeys + static_cast<size_t>(t) * E;
+  int e = -1;
+  if (lane < k) {
+    const int r = route_row[static_cast<size_t>(t) * k + lane];
+    e = (r >= 0) ? r / C : ids[static_cast<size_t>(t) * k + lane];
+  }
+  const bool valid = e >= 0 && e < E;
   const float zf = valid ? zrow[e] : -INFINITY;
   float g;
-  if (a.gate_mode != MOE_GATE_SOFTMAX_TOPK) {
+  if (gate_mode != MOE_GATE_SOFTMAX_TOPK) {
     // softmax over the final experts' logits.  For the renormalised mode this is
     // p_i / sum_j p_j with the full softmax's normaliser cancelled; shifting by the
     // final experts' own max keeps it finite when the token no longer holds its top
@@ -65,47 +85,58 @@ __device__ void regate(const AssignArgs& a, int t, const int* fin, int lane) {
     g = ex / warp_sum(ex);
   } else {  // the full-softmax probability of each final expert
     float m = -INFINITY;
-    for (int q = lane; q < a.E; q += 32) m = fmaxf(m, zrow[q]);
+    for (int q = lane; q < E; q += 32) m = fmaxf(m, zrow[q]);
     m = warp_max(m);
     float den = 0.f;
-    for (int q = lane; q < a.E; q += 32) den += expf(zrow[q] - m);
+    for (int q = lane; q < E; q += 32) den += expf(zrow[q] - m);
     den = warp_sum(den);
     g = valid ? expf(zf - m) / den : 0.f;
   }
-  if (lane < a.k) a.gates[static_cast<size_t>(t) * a.k + lane] = g;
+  if (lane < k) gates[static_cast<size_t>(t) * k + lane] = g;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) reroute_assign_kernel(AssignArgs a) {
-  __shared__ int s_cnt[256];
-  __shared__ int s_list[kThreads];
-  __shared__ int s_wtot[kWarps];
-  __shared__ uint32_t s_held[8];   // 256-bit set: experts the current token holds
-  __shared__ int s_fin[32];        // the current token's expert per slot
-  __shared__ int s_n, s_free, s_moved;
+// QE: experts per lane of the placing warp, ceil(E / 32) rounded up to a power of two.
+template <int QE>
+__global__ void __launch_bounds__(kAssignThreads, 1) reroute_assign_kernel(AssignArgs a) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  float* s_z = reinterpret_cast<float*>(smem);                                  // [chunk][E]
+  int* s_ids = reinterpret_cast<int*>(smem + static_cast<size_t>(a.chunk) * a.E * 4);  // [chunk][k]
+  __shared__ int s_list[kAssignThreads];
+  __shared__ int s_row[kAssignThreads];  // placed row of each listed route, -1 if none
+  __shared__ int s_mv[kAssignThreads];   // its index in the list of moved routes
+  __shared__ int s_wtot[kAssignWarps];
+  __shared__ int s_n, s_done;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = a.E, k = a.k, C = a.C;
-  pdl_trigger();
+  // The dependent launch is released only at the end (below): a dependent grid made
+  // resident early would share this CTA's SM while the placing warp runs.
   pdl_wait();  // route_row, counts and the keys come from the router and the pack
 
-  for (int e = tid; e < E; e += kThreads) s_cnt[e] = a.offsets[E + 2 + e];
-  __syncthreads();
+  // placing warp's state: counts and held flags of experts lane + 32 q
+  int cnt[QE];
+  bool held[QE];
+  int free_total = 0;
   if (warp == 0) {
     int f = 0;
-    for (int e = lane; e < E; e += 32) f += C - s_cnt[e];
 #pragma unroll
-    for (int s = 16; s >= 1; s >>= 1) f += __shfl_xor_sync(0xffffffffu, f, s);
-    if (lane == 0) { s_free = f; s_moved = 0; }
+    for (int q = 0; q < QE; ++q) {
+      const int e = lane + 32 * q;
+      cnt[q] = (e < E) ? a.offsets[E + 2 + e] : C;
+      held[q] = false;
+      f += C - cnt[q];
+    }
+    free_total = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(f)));
+    if (lane == 0) s_done = free_total <= 0 ? 1 : 0;
   }
   __syncthreads();
 
   const int total = a.T * k;  // <= INT_MAX / 2 (validated on the host)
-  int cur_t = -1;             // warp 0: token whose routes are being placed
-  bool cur_moved = false;
-  for (int base = 0; base < total && s_free > 0; base += kThreads) {
+  int cur_t = -1, moved = 0;
+  for (int base = 0; base < total && !s_done; base += a.chunk) {
     // 1. overflowed routes of this chunk, in arrival order
     const int r = base + tid;
     bool flag = false;
-    if (r < total) {
+    if (tid < a.chunk && r < total) {
       const int t = r / k, j = r - t * k;
       const int32_t* row = a.ids + static_cast<size_t>(t) * k;
       flag = a.route_row[r] < 0 && route_id_valid(row, j, row[j], E);
@@ -115,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1) reroute_assign_kernel(AssignArgs 
     __syncthreads();
     int before = 0, n = 0;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
+    for (int w = 0; w < kAssignWarps; ++w) {
       before += (w < warp) ? s_wtot[w] : 0;
       n += s_wtot[w];
     }
@@ -123,88 +154,108 @@ __global__ void __launch_bounds__(kThreads, 1) reroute_assign_kernel(AssignArgs 
     if (tid == 0) s_n = n;
     __syncthreads();
 
-    // 2. warp 0 places them one at a time
+    // 2. stage their tokens' ranking keys and expert ids
+    for (int idx = tid; idx < n * E; idx += kAssignThreads) {
+      const int i = idx / E, e = idx - i * E;
+      s_z[idx] = a.zkeys[static_cast<size_t>(s_list[i] / k) * E + e];
+    }
+    for (int idx = tid; idx < n * k; idx += kAssignThreads) {
+      const int i = idx / k, jj = idx - i * k;
+      s_ids[idx] = a.ids[static_cast<size_t>(s_list[i] / k) * k + jj];
+    }
+    if (tid < n) s_row[tid] = -1;
+    __syncthreads();
+
+    // 3. one warp places them in order
     if (warp == 0) {
-      for (int i = 0; i < s_n; ++i) {
-        __syncwarp();
-        if (s_free <= 0) break;
+      for (int i = 0; i < n; ++i) {
         const int rr = s_list[i];
-        const int t = rr / k, j = rr - t * k;
-        if (t != cur_t) {
-          if (cur_moved) regate(a, cur_t, s_fin, lane);
+        const int t = rr / k;
+        if (t != cur_t) {  // a new token: it holds its own top-k experts
           cur_t = t;
-          cur_moved = false;
-          if (lane < 8) s_held[lane] = 0u;
-          __syncwarp();
-          if (lane < k) {
-            const int e = a.ids[static_cast<size_t>(t) * k + lane];
-            s_fin[lane] = e;
-            if (e >= 0 && e < E) atomicOr(&s_held[e >> 5], 1u << (e & 31));
-          }
-          __syncwarp();
-        }
-        const float* zrow = a.zkeys + static_cast<size_t>(t) * E;
-        float bv = -INFINITY;
-        int be = INT_MAX;  // INT_MAX: no candidate
-        for (int e = lane; e < E; e += 32) {
-          if (((s_held[e >> 5] >> (e & 31)) & 1u) == 0u && s_cnt[e] < C) {
-            const float v = zrow[e];
-            if (be == INT_MAX || v > bv || (v == bv && e < be)) { bv = v; be = e; }
-          }
-        }
 #pragma unroll
-        for (int s = 16; s >= 1; s >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, bv, s);
-          const int oe = __shfl_xor_sync(0xffffffffu, be, s);
-          if (oe != INT_MAX && (be == INT_MAX || ov > bv || (ov == bv && oe < be))) {
-            bv = ov;
-            be = oe;
+          for (int q = 0; q < QE; ++q) held[q] = false;
+          for (int jj = 0; jj < k; ++jj) {
+            const int e0 = s_ids[i * k + jj];
+#pragma unroll
+            for (int q = 0; q < QE; ++q) held[q] = held[q] || (e0 == lane + 32 * q);
           }
         }
-        if (be != INT_MAX) {  // the same on every lane
-          if (lane == 0) {
-            const int slot = s_cnt[be];
-            s_cnt[be] = slot + 1;
-            const int row = be * C + slot;
-            a.route_row[rr] = row;
-            a.row_token[row] = t;
-            const int m = s_moved;
-            a.list[1 + 2 * m] = t;
-            a.list[2 + 2 * m] = row;
-            s_moved = m + 1;
-            s_free = s_free - 1;
-            s_fin[j] = be;
-            s_held[be >> 5] |= 1u << (be & 31);
+        uint32_t best = 0u;
+        unsigned best_e = 0xffffffffu;
+#pragma unroll
+        for (int q = 0; q < QE; ++q) {
+          const int e = lane + 32 * q;
+          if (e < E && !held[q] && cnt[q] < C) {
+            const uint32_t code = key_code(s_z[i * E + e]);
+            if (code > best) { best = code; best_e = static_cast<unsigned>(e); }
           }
-          cur_moved = true;
         }
+        const uint32_t m = __reduce_max_sync(0xffffffffu, best);
+        if (m == 0u) continue;  // no free expert the token does not hold: stays dropped
+        const int es = static_cast<int>(__reduce_min_sync(0xffffffffu, best == m ? best_e : 0xffffffffu));
+        const int owner = es & 31, qs = es >> 5;
+        int slot = 0;
+#pragma unroll
+        for (int q = 0; q < QE; ++q)
+          if (q == qs && lane == owner) { slot = cnt[q]; cnt[q] = slot + 1; held[q] = true; }
+        slot = __shfl_sync(0xffffffffu, slot, owner);
+        if (lane == 0) {  // results go out after the walk, written by the whole CTA
+          s_row[i] = es * C + slot;
+          s_mv[i] = moved;
+        }
+        ++moved;
+        if (--free_total == 0) break;
       }
-      __syncwarp();
+      if (lane == 0) s_done = free_total == 0 ? 1 : 0;
     }
     __syncthreads();
+    // 4. write this chunk's placements
+    if (tid < n && s_row[tid] >= 0) {
+      const int rr = s_list[tid], row = s_row[tid], m = s_mv[tid];
+      const int t = rr / k;
+      a.route_row[rr] = row;
+      a.row_token[row] = t;
+      a.list[1 + 2 * m] = t;
+      a.list[2 + 2 * m] = row;
+    }
   }
-  if (warp == 0 && cur_moved) regate(a, cur_t, s_fin, lane);
-  __syncthreads();
-  for (int e = tid; e < E; e += kThreads) a.offsets[E + 2 + e] = s_cnt[e];
-  if (tid == 0) a.list[0] = s_moved;
+  if (warp == 0) {
+#pragma unroll
+    for (int q = 0; q < QE; ++q)
+      if (lane + 32 * q < E) a.offsets[E + 2 + lane + 32 * q] = cnt[q];
+    if (lane == 0) a.list[0] = moved;
+  }
+  pdl_trigger();
 }
 
-// One warp per moved route: copy x[t] to its new row of the padded buffer.
+struct CopyArgs {
+  const void* x;
+  void* x_packed;
+  const int32_t* list;
+  const int32_t* ids;
+  const float* zkeys;
+  const int32_t* route_row;
+  float* gates;
+  int d, k, E, C, gate_mode;
+};
+
+// One warp per moved route: copy x[t] to its new row of the padded buffer and re-evaluate
+// token t's gates (a token with two moved routes is evaluated twice, to the same values).
 template <typename T>
-__global__ void __launch_bounds__(kThreads) reroute_copy_kernel(const T* __restrict__ x,
-                                                                T* __restrict__ xp,
-                                                                const int32_t* list, int d) {
+__global__ void __launch_bounds__(kThreads) reroute_copy_kernel(CopyArgs a) {
   constexpr int VEC = Vec<T>::N;
   pdl_trigger();
   pdl_wait();
-  const int n = list[0];
+  const int n = a.list[0];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nvec = d / VEC;
+  const int nvec = a.d / VEC;
   for (int i = blockIdx.x * kWarps + warp; i < n; i += gridDim.x * kWarps) {
-    const int t = list[1 + 2 * i], row = list[2 + 2 * i];
-    const T* src = x + static_cast<size_t>(t) * d;
-    T* dst = xp + static_cast<size_t>(row) * d;
+    const int t = a.list[1 + 2 * i], row = a.list[2 + 2 * i];
+    const T* src = static_cast<const T*>(a.x) + static_cast<size_t>(t) * a.d;
+    T* dst = static_cast<T*>(a.x_packed) + static_cast<size_t>(row) * a.d;
     for (int v = lane; v < nvec; v += 32) st_vec(dst + v * VEC, ld_vec(src + v * VEC));
+    regate(a.ids, a.zkeys, a.route_row, a.gates, t, a.k, a.E, a.C, a.gate_mode, lane);
   }
 }
 
@@ -215,21 +266,39 @@ cudaError_t launch_reroute(const moe_config& c, const void* x, const int32_t* id
                            int32_t* route_row, int32_t* offsets, int32_t* list, int32_t* status,
                            cudaStream_t s) {
   (void)status;
-  AssignArgs a{ids, zkeys, gates, row_token, route_row, offsets, list,
-               c.T, c.k, c.E, c.capacity, c.gate_mode};
-  cudaError_t e = launch_pdl(reroute_assign_kernel, dim3(1), dim3(kThreads), 0, s, a);
+  int chunk = kAssignThreads;
+  if (chunk > kStageFloats / c.E) chunk = kStageFloats / c.E;
+  if (chunk > kStageIds / c.k) chunk = kStageIds / c.k;
+  AssignArgs a{ids, zkeys, row_token, route_row, offsets, list, c.T, c.k, c.E, c.capacity, chunk};
+  const size_t smem = static_cast<size_t>(chunk) * (c.E + c.k) * 4;
+  static bool configured = false;
+  if (!configured) {
+    const int lim = (kStageFloats + kStageIds) * 4;
+    cudaFuncSetAttribute(reroute_assign_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+    cudaFuncSetAttribute(reroute_assign_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+    cudaFuncSetAttribute(reroute_assign_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+    cudaFuncSetAttribute(reroute_assign_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+    configured = true;
+  }
+  cudaError_t e;
+  if (c.E <= 32)
+    e = launch_pdl(reroute_assign_kernel<1>, dim3(1), dim3(kAssignThreads), smem, s, a);
+  else if (c.E <= 64)
+    e = launch_pdl(reroute_assign_kernel<2>, dim3(1), dim3(kAssignThreads), smem, s, a);
+  else if (c.E <= 128)
+    e = launch_pdl(reroute_assign_kernel<4>, dim3(1), dim3(kAssignThreads), smem, s, a);
+  else
+    e = launch_pdl(reroute_assign_kernel<8>, dim3(1), dim3(kAssignThreads), smem, s, a);
   if (e != cudaSuccess) return e;
   long long slots = static_cast<long long>(c.E) * c.capacity;
   int grid = static_cast<int>((slots + kWarps - 1) / kWarps);
   if (grid > 4 * 148) grid = 4 * 148;
   if (grid < 1) grid = 1;
+  const CopyArgs ca{x, x_packed, list, ids, zkeys, route_row, gates, c.d, c.k, c.E, c.capacity,
+                    c.gate_mode};
   if (c.dtype == MOE_BF16)
-    return launch_pdl(reroute_copy_kernel<__nv_bfloat16>, dim3(grid), dim3(kThreads), 0, s,
-                      static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(x_packed),
-                      static_cast<const int32_t*>(list), c.d);
-  return launch_pdl(reroute_copy_kernel<float>, dim3(grid), dim3(kThreads), 0, s,
-                    static_cast<const float*>(x), static_cast<float*>(x_packed),
-                    static_cast<const int32_t*>(list), c.d);
+    return launch_pdl(reroute_copy_kernel<__nv_bfloat16>, dim3(grid), dim3(kThreads), 0, s, ca);
+  return launch_pdl(reroute_copy_kernel<float>, dim3(grid), dim3(kThreads), 0, s, ca);
 }
 
 }  // namespace moe

@@ -38,6 +38,8 @@ class Workload:
     layers: int = 1
     router_std: float | None = 0.02    # None: d ** -0.5
     expert_std: float | None = 0.02    # None: d ** -0.5
+    layout: str = "ragged"             # ragged | padded ([E, C, d] buffer; needs phi)
+    overflow: str = "drop"             # drop | reroute (padded only)
     bias: str = "none"                 # none | switch | zipf | normal
 
     def with_(self, **kw) -> "Workload":
@@ -76,6 +78,14 @@ for _T in (1, 16, 256, 4096):
             f"shared64_T{_T}_{_tag}", T=_T, d=4096, E=64, k=2, d_ff=32768,
             gate_mode="softmax_topk_renorm", phi=_phi, has_shared=True, router_std=None,
             bias="normal")
+
+
+# The Switch-shaped and 64+1 layers with capacity through the padded [E, C, d] buffer and
+# the reroute overflow policy.
+WORKLOADS["switch_phi125_reroute"] = WORKLOADS["switch_phi125"].with_(
+    name="switch_phi125_reroute", layout="padded", overflow="reroute")
+WORKLOADS["shared64_T4096_phi1_reroute"] = WORKLOADS["shared64_T4096_phi1"].with_(
+    name="shared64_T4096_phi1_reroute", layout="padded", overflow="reroute")
 
 
 def _randn(shape, gen, device, std, dtype):

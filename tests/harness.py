@@ -25,7 +25,7 @@ def config_for(wl: I.Workload, capacity=None, stats=False) -> N.MoeConfig:
         capacity = -1 if wl.phi is None else N.moe_capacity(wl.T, wl.k, wl.E, *wl.phi)
     return N.make_config(wl.T, wl.d, wl.E, wl.k, wl.d_ff, dtype=wl.dtype, gate_mode=wl.gate_mode,
                          capacity=capacity, has_shared=wl.has_shared, add_residual=wl.add_residual,
-                         stats=stats)
+                         stats=stats, layout=wl.layout, overflow=wl.overflow)
 
 
 def oracle_params(p: dict) -> dict:
