@@ -363,6 +363,306 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 5) tmem_dealloc(tmem_base, p.tmem_cols);
 }
 
+// ---------------------------------------------------------------------------------
+// Cluster variant (E <= 64, d >= 8 * 64): the 128-token tile is shared by a cluster of 8
+// CTAs.  CTA r contracts d-blocks [r KB / 8, (r+1) KB / 8) for all 128 tokens, so the tile's
+// x streams through 8 SMs instead of one.  The 8 partial logit tiles meet in distributed
+// shared memory: CTA r adds up the rows of its 16 tokens from all 8 CTAs in rank order
+// (the same order every run), adds the bias, and runs the epilogue with 8 lanes per token:
+// k rounds of a 3-step arg-max within the 8-lane group (larger logit, then lower expert
+// index).  CTA 0 adds up the 8 per-CTA histograms (and probability sums) in rank order.
+// ---------------------------------------------------------------------------------
+constexpr int kCluster = 8;
+constexpr int kMaxSmemPerCta = 227 * 1024;
+constexpr int kTokPerCta = kTokens / kCluster;  // 16
+constexpr int kLanesPerTok = 128 / kTokPerCta;  // 8
+
+template <int EN_T, int KMAX>
+__global__ void __launch_bounds__(kThreads, 1)
+    router_cluster_kernel(const __grid_constant__ RouteMaps maps, const RouteParams p) {
+  constexpr int V = EN_T / kLanesPerTok;  // logits per lane
+  static_assert(V >= 1 && V <= 32, "logits per lane");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int stage_bytes = A_BYTES + EN_T * BK * 2;
+  float* s_part = reinterpret_cast<float*>(base + p.stages * stage_bytes);  // [128][EN_T]
+  float* s_red = s_part + kTokens * EN_T;                                   // [16][EN_T]
+  float* s_p = s_red + kTokPerCta * EN_T;                                   // [16][EN_T]
+  uint8_t* ctl = reinterpret_cast<uint8_t*>(s_p + kTokPerCta * EN_T);
+  uint64_t* full = reinterpret_cast<uint64_t*>(ctl);
+  uint64_t* empty = full + kMaxStages;
+  uint64_t* tfull = empty + kMaxStages;
+  uint64_t* drain = tfull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 8 * (2 * kMaxStages + 2));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* s_bias = reinterpret_cast<float*>(ctl + 256);
+  int* s_hist = reinterpret_cast<int*>(ctl + 256 + 256 * 4);
+  float* s_psum = reinterpret_cast<float*>(ctl + 256 + 2 * 256 * 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int tile = blockIdx.x / kCluster;
+  const int KB = p.d / BK;
+  const int kb0 = static_cast<int>(rank) * KB / kCluster;
+  const int kb1 = (static_cast<int>(rank) + 1) * KB / kCluster;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    mbar_init(tfull, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&maps.x);
+    tma_prefetch_desc(&maps.w);
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, p.tmem_cols);
+    tmem_relinquish();
+  }
+  pdl_trigger();
+  pdl_wait();  // x comes from the previous layer; ids/gates/hist are read by earlier kernels
+  for (int e = threadIdx.x; e < 256; e += kThreads) {
+    s_bias[e] = (e < p.E && p.bias != nullptr) ? __ldg(p.bias + e) : 0.f;
+    s_hist[e] = 0;
+    s_psum[e] = 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 4 && lane == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    bool wrapped = false, ok = true;
+    for (int kb = kb0; kb < kb1; ++kb) {
+      if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.limit_ns, p.status)) {
+        ok = false;
+        break;
+      }
+      mbar_arrive_expect_tx(&full[stage], stage_bytes);
+      uint8_t* dst = base + stage * stage_bytes;
+      tma_load_2d(dst, &maps.x, &full[stage], kb * BK, tile * kTokens);
+      tma_load_2d(dst + A_BYTES, &maps.w, &full[stage], kb * BK, 0);
+      if (++stage == p.stages) { stage = 0; phase ^= 1u; wrapped = true; }
+    }
+    if (!ok) {
+      for (int s = 0; s < p.stages; ++s) {
+        if (!wrapped && s >= stage) continue;
+        mbar_wait_bounded(&full[s], (s < stage) ? phase : (phase ^ 1u), nullptr, p.limit_ns, p.status);
+      }
+    }
+  } else if (warp == 5 && lane == 0) {
+    // ---------------------------------------------------------------- MMA issuer
+    const uint32_t idesc = idesc_bf16_f32(kTokens, EN_T);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int kb = kb0; kb < kb1; ++kb) {
+      if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.limit_ns, p.status)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint8_t* src = base + stage * stage_bytes;
+      const uint64_t ad = smem_desc_k_sw128(src);
+      const uint64_t bd = smem_desc_k_sw128(src + A_BYTES);
+#pragma unroll
+      for (int kk = 0; kk < BK / 16; ++kk)
+        tc_mma_bf16(tmem_base, ad + 2 * kk, bd + 2 * kk, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
+      tc_commit(&empty[stage]);
+      if (++stage == p.stages) { stage = 0; phase ^= 1u; }
+    }
+    if (ok) {
+      tc_commit(tfull);
+    } else {
+      tc_commit(drain);
+      mbar_wait_bounded(drain, 0, nullptr, p.limit_ns, p.status);
+    }
+  } else if (warp < 4) {
+    // ---------------------------------------------------------------- partial logits
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait_bounded(tfull, 0, abort_flag, p.limit_ns, p.status);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    float4* dst = reinterpret_cast<float4*>(s_part + (warp * 32 + lane) * EN_T);
+    if (ok) {
+      tc_fence_after();
+      const uint32_t trow = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+#pragma unroll
+      for (int c0 = 0; c0 < EN_T; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(trow + c0, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          dst[c0 / 4 + q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                                        __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < EN_T / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  __syncthreads();
+  cluster_sync_all();  // every CTA's partial logits are visible to the cluster
+
+  // ------------------------------------------------------------------ reduce my 16 tokens
+  const int row0 = static_cast<int>(rank) * kTokPerCta;
+  for (int c = threadIdx.x; c < kTokPerCta * EN_T / 4; c += kThreads) {
+    const int rl = c / (EN_T / 4), c4 = c - rl * (EN_T / 4);
+    const float* src = s_part + (row0 + rl) * EN_T + c4 * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int r = 0; r < kCluster; ++r) {
+      const float4 v = ld_cluster_f4(cluster_map(src, static_cast<uint32_t>(r)));
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e = c4 * 4 + q;
+      s_red[rl * EN_T + e] = (e < p.E) ? rank_key(a4[q] + s_bias[e]) : -INFINITY;
+    }
+  }
+  __syncthreads();
+
+  if (warp < 4) {
+    // ---------------------------------------------------------------- epilogue
+    const int tl = threadIdx.x / kLanesPerTok, g = threadIdx.x % kLanesPerTok;
+    const int t = tile * kTokens + row0 + tl;
+    float v[V];
+    uint32_t taken = 0;  // bit q: expert q * 8 + g is selected (or is padding past E)
+#pragma unroll
+    for (int q = 0; q < V; ++q) {
+      const int e = q * kLanesPerTok + g;
+      v[q] = s_red[tl * EN_T + e];
+      if (e >= p.E) taken |= 1u << q;
+    }
+    if (p.zkeys != nullptr && t < p.T) {
+#pragma unroll
+      for (int q = 0; q < V; ++q) {
+        const int e = q * kLanesPerTok + g;
+        if (e < p.E) p.zkeys[static_cast<size_t>(t) * p.E + e] = v[q];
+      }
+    }
+    float tv[KMAX];
+    int te[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      tv[j] = -INFINITY;
+      te[j] = 0;
+      if (j >= p.k) continue;
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int q = 0; q < V; ++q) {
+        const int e = q * kLanesPerTok + g;
+        if (!((taken >> q) & 1u) && (v[q] > bv || (v[q] == bv && e < be))) { bv = v[q]; be = e; }
+      }
+#pragma unroll
+      for (int s = kLanesPerTok / 2; s >= 1; s >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, s);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, s);
+        if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+      }
+      if (be < EN_T && be % kLanesPerTok == g) taken |= 1u << (be / kLanesPerTok);
+      tv[j] = bv;
+      te[j] = be;
+    }
+    const float m = tv[0];  // largest logit
+    const bool want_all = p.gate_mode != MOE_GATE_TOPK_SOFTMAX || p.tile_psum != nullptr;
+    float denom_all = 0.f;
+    if (want_all) {
+#pragma unroll
+      for (int q = 0; q < V; ++q)
+        if (q * kLanesPerTok + g < p.E) denom_all += expf(v[q] - m);
+#pragma unroll
+      for (int s = kLanesPerTok / 2; s >= 1; s >>= 1)
+        denom_all += __shfl_xor_sync(0xffffffffu, denom_all, s);
+    }
+    float gt[KMAX];
+    float sel = 0.f;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      gt[j] = (j < p.k) ? expf(tv[j] - m) : 0.f;
+      if (p.gate_mode != MOE_GATE_TOPK_SOFTMAX) gt[j] = gt[j] / denom_all;  // probability
+      sel += gt[j];
+    }
+    if (t < p.T) {
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        if (j < p.k && j % kLanesPerTok == g) {
+          const float gj = (p.gate_mode == MOE_GATE_SOFTMAX_TOPK) ? gt[j] : gt[j] / sel;
+          p.ids[static_cast<size_t>(t) * p.k + j] = te[j];
+          p.gates[static_cast<size_t>(t) * p.k + j] = gj;
+          atomicAdd(&s_hist[te[j]], 1);
+        }
+      }
+    }
+    if (p.tile_psum != nullptr) {
+      const float inv = (t < p.T) ? 1.f / denom_all : 0.f;
+#pragma unroll
+      for (int q = 0; q < V; ++q) {
+        const int e = q * kLanesPerTok + g;
+        s_p[tl * EN_T + e] = (e < p.E) ? expf(v[q] - m) * inv : 0.f;
+      }
+    }
+  }
+  __syncthreads();
+  if (p.tile_psum != nullptr && threadIdx.x < EN_T) {
+    float a = 0.f;
+    for (int tl = 0; tl < kTokPerCta; ++tl) a += s_p[tl * EN_T + threadIdx.x];
+    s_psum[threadIdx.x] = a;
+  }
+  cluster_sync_all();  // every CTA's histogram and probability sums are visible
+  if (rank == 0) {
+    for (int e = threadIdx.x; e < p.E; e += kThreads) {
+      int h = 0;
+      float ps = 0.f;
+      for (int r = 0; r < kCluster; ++r) {
+        h += ld_cluster_s32(cluster_map(&s_hist[e], static_cast<uint32_t>(r)));
+        if (p.tile_psum != nullptr) ps += ld_cluster_f32(cluster_map(&s_psum[e], static_cast<uint32_t>(r)));
+      }
+      if (p.tile_hist != nullptr) p.tile_hist[static_cast<size_t>(tile) * p.E + e] = h;
+      if (p.tile_psum != nullptr) p.tile_psum[static_cast<size_t>(tile) * p.E + e] = ps;
+    }
+  }
+  cluster_sync_all();  // CTA 0 has read the others' shared memory before any of them exits
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc(tmem_base, p.tmem_cols);
+}
+
+template <int EN_T, int KMAX>
+cudaError_t launch_cluster_kmax(const RouteMaps& maps, const RouteParams& p, int grid, int smem,
+                                cudaStream_t s) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(router_cluster_kernel<EN_T, KMAX>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmemPerCta);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  return launch_pdl_cluster(router_cluster_kernel<EN_T, KMAX>, dim3(grid), dim3(kThreads), smem,
+                            kCluster, s, maps, p);
+}
+
+template <int EN_T>
+cudaError_t launch_cluster_en(const RouteMaps& maps, const RouteParams& p, int grid, int smem,
+                              cudaStream_t s) {
+  if (p.k <= 1) return launch_cluster_kmax<EN_T, 1>(maps, p, grid, smem, s);
+  if (p.k <= 2) return launch_cluster_kmax<EN_T, 2>(maps, p, grid, smem, s);
+  if (p.k <= 4) return launch_cluster_kmax<EN_T, 4>(maps, p, grid, smem, s);
+  if (p.k <= 8) return launch_cluster_kmax<EN_T, 8>(maps, p, grid, smem, s);
+  if (p.k <= 16) return launch_cluster_kmax<EN_T, 16>(maps, p, grid, smem, s);
+  return launch_cluster_kmax<EN_T, 32>(maps, p, grid, smem, s);
+}
+
 template <int EN_T, int KMAX>
 cudaError_t launch_kmax(const RouteMaps& maps, const RouteParams& p, int grid, int smem,
                         cudaStream_t s) {
@@ -412,7 +712,22 @@ cudaError_t launch_router_sm100(const moe_config& c, const void* x, const void* 
     return cudaErrorInvalidValue;
   RouteParams p{bias, c.T, c.d, c.E, c.k, EN, c.gate_mode, stages, cols,
                 ids, gates, tile_hist, tile_psum, extra.zkeys, status, kWaitLimitNs};
-  const int grid = (c.T + kTokens - 1) / kTokens;
+  const int ntiles = (c.T + kTokens - 1) / kTokens;
+  if (EN <= 64 && k_blocks >= kCluster) {
+    // one 128-token tile per cluster of 8 CTAs, each with 1/8 of d
+    const int fixed = 1024 + (kTokens + 2 * kTokPerCta) * EN * 4 + 256 + 3 * 256 * 4;
+    int cstages = (k_blocks + kCluster - 1) / kCluster;
+    if (cstages > stages) cstages = stages;
+    if (cstages > (kMaxSmemPerCta - fixed) / stage_bytes) cstages = (kMaxSmemPerCta - fixed) / stage_bytes;
+    RouteParams pc = p;
+    pc.stages = cstages;
+    const int csmem = fixed + cstages * stage_bytes;
+    const int cgrid = ntiles * kCluster;
+    if (EN == 16) return launch_cluster_en<16>(maps, pc, cgrid, csmem, s);
+    if (EN == 32) return launch_cluster_en<32>(maps, pc, cgrid, csmem, s);
+    return launch_cluster_en<64>(maps, pc, cgrid, csmem, s);
+  }
+  const int grid = ntiles;
   const int smem = 1024 + stages * stage_bytes + 256 + 2 * 256 * 4 + (tile_psum ? 4 * 256 * 4 : 0);
   if (EN == 16) return launch_en<16>(maps, p, grid, smem, s);
   if (EN == 32) return launch_en<32>(maps, p, grid, smem, s);
