@@ -75,6 +75,7 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
   __shared__ int s_off[257];   // segment starts over kept routes
   __shared__ int s_rows[kSubTok][32];
   __shared__ uint32_t s_mask[256 * kWords];  // [E][words]: bit = token of the tile chose e
+  __shared__ int s_ids[kHistTile * 32];      // the histogram tile's expert ids [128][k]
   __shared__ __align__(8) uint64_t s_bar;
   extern __shared__ __align__(128) uint8_t s_stage[];  // copy_round token rows
 
@@ -90,6 +91,25 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
   for (int w = tid; w < E * kWords; w += kThreads) s_mask[w] = 0;
   pdl_trigger();
   pdl_wait();
+
+  // 0. The token rows do not depend on the routing: start the first round of their bulk
+  //    loads now, so that they arrive while the positions are being worked out.
+  const uint32_t row_bytes = static_cast<uint32_t>(a.d) * sizeof(T);
+  const int round = a.copy_round;  // token rows staged at a time
+  const T* __restrict__ X = static_cast<const T*>(a.x);
+  T* __restrict__ XP = static_cast<T*>(a.x_packed);
+  if (tid == 0) {
+    mbar_init(&s_bar, 1);
+    fence_mbar_init();
+    const int nr = min(round, nsub);
+    mbar_arrive_expect_tx(&s_bar, nr * row_bytes);
+    for (int i = 0; i < nr; ++i)
+      bulk_load(s_stage + i * row_bytes, X + static_cast<size_t>(t_begin + i) * a.d, row_bytes,
+                &s_bar);
+  }
+  // The tile's expert ids, one coalesced pass (its loads overlap the histogram's below).
+  for (int r = tid; r < ntile * k; r += kThreads)
+    s_ids[r] = __ldg(a.ids + static_cast<size_t>(tile0) * k + r);
   __syncthreads();
 
   // 1. prefix (tiles < this one) and total per expert, split over all threads with
@@ -119,7 +139,7 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
   // 2. bitmask of the histogram tile's tokens per expert
   for (int r = tid; r < ntile * k; r += kThreads) {
     const int tl = r / k, j = r % k;
-    const int32_t* row = a.ids + static_cast<size_t>(tile0 + tl) * k;
+    const int32_t* row = s_ids + tl * k;
     const int e = row[j];
     if (route_id_valid(row, j, e, E)) atomicOr(&s_mask[e * kWords + (tl >> 5)], 1u << (tl & 31));
   }
@@ -168,7 +188,7 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
   for (int r = tid; r < nsub * k; r += kThreads) {
     const int ts = r / k, j = r - ts * k;
     const int t = t_begin + ts, tl = t - tile0;
-    const int32_t* row = a.ids + static_cast<size_t>(t) * k;
+    const int32_t* row = s_ids + tl * k;
     const int e = row[j];
     int out = -1;
     if (route_id_valid(row, j, e, E)) {
@@ -189,24 +209,17 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
   // 5. copy with the bulk-copy engine: each token row is loaded once into shared memory
   //    and stored once per kept route (warp 0 issues; the engine moves whole rows)
   if (warp != 0) return;
-  const uint32_t row_bytes = static_cast<uint32_t>(a.d) * sizeof(T);
-  const int round = a.copy_round;  // token rows staged at a time
-  const T* __restrict__ X = static_cast<const T*>(a.x);
-  T* __restrict__ XP = static_cast<T*>(a.x_packed);
-  if (lane == 0) {
-    mbar_init(&s_bar, 1);
-    fence_mbar_init();
-  }
-  __syncwarp();
   uint32_t phase = 0;
   for (int r0 = 0; r0 < nsub; r0 += round) {
     const int nr = min(round, nsub - r0);
     int ok = 1;
     if (lane == 0) {
-      mbar_arrive_expect_tx(&s_bar, nr * row_bytes);
-      for (int i = 0; i < nr; ++i)
-        bulk_load(s_stage + i * row_bytes, X + static_cast<size_t>(t_begin + r0 + i) * a.d, row_bytes,
-                  &s_bar);
+      if (r0 > 0) {  // the first round was issued at the start
+        mbar_arrive_expect_tx(&s_bar, nr * row_bytes);
+        for (int i = 0; i < nr; ++i)
+          bulk_load(s_stage + i * row_bytes, X + static_cast<size_t>(t_begin + r0 + i) * a.d,
+                    row_bytes, &s_bar);
+      }
       ok = mbar_wait_bounded(&s_bar, phase, nullptr, kWaitLimitNs, a.status);
       if (!ok) mbar_wait_bounded(&s_bar, phase, nullptr, kWaitLimitNs, a.status);  // drain
     }
@@ -219,7 +232,9 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
       if (r >= 0) bulk_store(XP + static_cast<size_t>(r) * a.d, s_stage + i * row_bytes, row_bytes);
     }
     bulk_commit();
-    bulk_wait_all();  // the stage is reused next round; the rows are written before exit
+    // The stage is reused by the next round, and must outlive the stores' reads of it
+    // before the CTA exits; the stores then complete on their own.
+    bulk_wait_read_all();
     __syncwarp();
   }
 }

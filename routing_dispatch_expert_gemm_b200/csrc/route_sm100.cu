@@ -165,10 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   pdl_trigger();
   pdl_wait();  // x comes from the previous layer; ids/gates/hist are read by earlier kernels
-  for (int e = threadIdx.x; e < 256; e += kThreads) {
-    s_bias[e] = (e < p.E && p.bias != nullptr) ? __ldg(p.bias + e) : 0.f;
-    s_hist[e] = 0;
-  }
+  for (int e = threadIdx.x; e < 256; e += kThreads) s_hist[e] = 0;
   if (p.tile_psum != nullptr)
     for (int i = threadIdx.x; i < 4 * 256; i += kThreads) s_psum[i] = 0.f;
   tc_fence_before();
@@ -227,6 +224,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 4) {
     // ---------------------------------------------------------------- epilogue
+    // The bias is read while the contraction runs (epilogue threads only).
+    for (int e = threadIdx.x; e < 256; e += 128)
+      s_bias[e] = (e < p.E && p.bias != nullptr) ? __ldg(p.bias + e) : 0.f;
+    epilogue_bar();
     int ok = 1;
     if (lane == 0) ok = mbar_wait_bounded(tfull, 0, abort_flag, p.limit_ns, p.status);
     ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -425,7 +426,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_trigger();
   pdl_wait();  // x comes from the previous layer; ids/gates/hist are read by earlier kernels
   for (int e = threadIdx.x; e < 256; e += kThreads) {
-    s_bias[e] = (e < p.E && p.bias != nullptr) ? __ldg(p.bias + e) : 0.f;
     s_hist[e] = 0;
     s_psum[e] = 0.f;
   }
@@ -485,6 +485,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 4) {
     // ---------------------------------------------------------------- partial logits
+    // (the bias is read here, off the producer's critical path; it is used after the
+    // block barrier below)
+    for (int e = threadIdx.x; e < 256; e += 128)
+      s_bias[e] = (e < p.E && p.bias != nullptr) ? __ldg(p.bias + e) : 0.f;
     int ok = 1;
     if (lane == 0) ok = mbar_wait_bounded(tfull, 0, abort_flag, p.limit_ns, p.status);
     ok = __shfl_sync(0xffffffffu, ok, 0);
