@@ -370,8 +370,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // x streams through 8 SMs instead of one.  The 8 partial logit tiles meet in distributed
 // shared memory: CTA r adds up the rows of its 16 tokens from all 8 CTAs in rank order
 // (the same order every run), adds the bias, and runs the epilogue with 8 lanes per token:
-// k rounds of a 3-step arg-max within the 8-lane group (larger logit, then lower expert
-// index).  CTA 0 adds up the 8 per-CTA histograms (and probability sums) in rank order.
+// each lane counts the rank of its experts against the token's row (larger logit first, then
+// lower expert index) and writes the ones ranked below k to their slots.  CTA 0 adds up the
+// 8 per-CTA histograms (and probability sums) in rank order.
 // ---------------------------------------------------------------------------------
 constexpr int kCluster = 8;
 constexpr int kMaxSmemPerCta = 227 * 1024;
@@ -400,6 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* s_bias = reinterpret_cast<float*>(ctl + 256);
   int* s_hist = reinterpret_cast<int*>(ctl + 256 + 256 * 4);
   float* s_psum = reinterpret_cast<float*>(ctl + 256 + 2 * 256 * 4);
+  float* s_gsel = reinterpret_cast<float*>(ctl + 256 + 3 * 256 * 4);  // [16][32] top-k exps
+  float* s_gden = s_gsel + kTokPerCta * 32;                           // [16][8] partial sums
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
@@ -553,57 +556,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (e < p.E) p.zkeys[static_cast<size_t>(t) * p.E + e] = v[q];
       }
     }
-    float tv[KMAX];
-    int te[KMAX];
+    // Rank of each of my experts in the token's order (logit descending, then expert index
+    // ascending), counted against the token's whole row, which the 8 lanes read from
+    // shared memory as a broadcast: rank r < k means slot r.  The row maximum is the
+    // top logit.
+    const float* zrow = s_red + tl * EN_T;
+    int rk[V];
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      tv[j] = -INFINITY;
-      te[j] = 0;
-      if (j >= p.k) continue;
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
+    for (int q = 0; q < V; ++q) rk[q] = 0;
+    float m = -INFINITY;
+#pragma unroll 8
+    for (int e2 = 0; e2 < EN_T; ++e2) {
+      const float z2 = zrow[e2];
+      m = fmaxf(m, z2);
 #pragma unroll
       for (int q = 0; q < V; ++q) {
         const int e = q * kLanesPerTok + g;
-        if (!((taken >> q) & 1u) && (v[q] > bv || (v[q] == bv && e < be))) { bv = v[q]; be = e; }
+        rk[q] += (z2 > v[q] || (z2 == v[q] && e2 < e)) ? 1 : 0;
       }
-#pragma unroll
-      for (int s = kLanesPerTok / 2; s >= 1; s >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, s);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, s);
-        if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-      }
-      if (be < EN_T && be % kLanesPerTok == g) taken |= 1u << (be / kLanesPerTok);
-      tv[j] = bv;
-      te[j] = be;
     }
-    const float m = tv[0];  // largest logit
-    const bool want_all = p.gate_mode != MOE_GATE_TOPK_SOFTMAX || p.tile_psum != nullptr;
+    // The token's exps of the selected logits go to their slots, and the lanes' partial sums
+    // of all exps to their places; both are then added up in a fixed order (slot order for
+    // the selected total) by every lane of the token.
+    float ex[V];
+    float dpart = 0.f;
+#pragma unroll
+    for (int q = 0; q < V; ++q) {
+      const int e = q * kLanesPerTok + g;
+      ex[q] = (e < p.E) ? expf(v[q] - m) : 0.f;
+      dpart += ex[q];
+      if (e < p.E && rk[q] < p.k) s_gsel[tl * 32 + rk[q]] = ex[q];
+    }
+    s_gden[tl * kLanesPerTok + g] = dpart;
+    __syncwarp();
     float denom_all = 0.f;
-    if (want_all) {
 #pragma unroll
-      for (int q = 0; q < V; ++q)
-        if (q * kLanesPerTok + g < p.E) denom_all += expf(v[q] - m);
-#pragma unroll
-      for (int s = kLanesPerTok / 2; s >= 1; s >>= 1)
-        denom_all += __shfl_xor_sync(0xffffffffu, denom_all, s);
-    }
-    float gt[KMAX];
+    for (int g2 = 0; g2 < kLanesPerTok; ++g2) denom_all += s_gden[tl * kLanesPerTok + g2];
+    const bool prob = p.gate_mode != MOE_GATE_TOPK_SOFTMAX;  // gates are probabilities first
     float sel = 0.f;
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      gt[j] = (j < p.k) ? expf(tv[j] - m) : 0.f;
-      if (p.gate_mode != MOE_GATE_TOPK_SOFTMAX) gt[j] = gt[j] / denom_all;  // probability
-      sel += gt[j];
-    }
+    for (int j = 0; j < p.k; ++j) sel += prob ? s_gsel[tl * 32 + j] / denom_all : s_gsel[tl * 32 + j];
     if (t < p.T) {
 #pragma unroll
-      for (int j = 0; j < KMAX; ++j) {
-        if (j < p.k && j % kLanesPerTok == g) {
-          const float gj = (p.gate_mode == MOE_GATE_SOFTMAX_TOPK) ? gt[j] : gt[j] / sel;
-          p.ids[static_cast<size_t>(t) * p.k + j] = te[j];
-          p.gates[static_cast<size_t>(t) * p.k + j] = gj;
-          atomicAdd(&s_hist[te[j]], 1);
+      for (int q = 0; q < V; ++q) {
+        const int e = q * kLanesPerTok + g;
+        if (e < p.E && rk[q] < p.k) {
+          const float gp = prob ? ex[q] / denom_all : ex[q];
+          const float gj = (p.gate_mode == MOE_GATE_SOFTMAX_TOPK) ? gp : gp / sel;
+          p.ids[static_cast<size_t>(t) * p.k + rk[q]] = e;
+          p.gates[static_cast<size_t>(t) * p.k + rk[q]] = gj;
+          atomicAdd(&s_hist[e], 1);
         }
       }
     }
@@ -719,7 +720,8 @@ cudaError_t launch_router_sm100(const moe_config& c, const void* x, const void* 
   const int ntiles = (c.T + kTokens - 1) / kTokens;
   if (EN <= 64 && k_blocks >= kCluster) {
     // one 128-token tile per cluster of 8 CTAs, each with 1/8 of d
-    const int fixed = 1024 + (kTokens + 2 * kTokPerCta) * EN * 4 + 256 + 3 * 256 * 4;
+    const int fixed = 1024 + (kTokens + 2 * kTokPerCta) * EN * 4 + 256 + 3 * 256 * 4 +
+                      kTokPerCta * (32 + kLanesPerTok) * 4;
     int cstages = (k_blocks + kCluster - 1) / kCluster;
     if (cstages > stages) cstages = stages;
     if (cstages > (kMaxSmemPerCta - fixed) / stage_bytes) cstages = (kMaxSmemPerCta - fixed) / stage_bytes;
