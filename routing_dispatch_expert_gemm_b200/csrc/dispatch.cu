@@ -67,7 +67,6 @@ constexpr size_t kStageBudget = 64 * 1024;  // shared memory staging token rows 
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
-  constexpr int VEC = Vec<T>::N;
   constexpr int kBatch = 8;    // histogram loads in flight per thread
   constexpr int kWords = kHistTile / 32;
   __shared__ int s_pre[256];   // routes to e in earlier tiles
@@ -206,36 +205,39 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
   }
   __syncthreads();
 
-  // 5. copy with the bulk-copy engine: each token row is loaded once into shared memory
-  //    and stored once per kept route (warp 0 issues; the engine moves whole rows)
-  if (warp != 0) return;
+  // 5. copy: each token row is loaded once into shared memory by the bulk-copy engine
+  //    (the first round was issued at the start) and written to each of its kept routes'
+  //    rows by all warps with 16-byte stores, one warp per destination row.
+  __shared__ int s_ok;
   uint32_t phase = 0;
+  const int nvec = static_cast<int>(row_bytes / 16);
   for (int r0 = 0; r0 < nsub; r0 += round) {
     const int nr = min(round, nsub - r0);
-    int ok = 1;
-    if (lane == 0) {
-      if (r0 > 0) {  // the first round was issued at the start
+    if (r0 > 0) {
+      __syncthreads();  // every warp has finished reading the previous round's rows
+      if (tid == 0) {
         mbar_arrive_expect_tx(&s_bar, nr * row_bytes);
         for (int i = 0; i < nr; ++i)
           bulk_load(s_stage + i * row_bytes, X + static_cast<size_t>(t_begin + r0 + i) * a.d,
                     row_bytes, &s_bar);
       }
-      ok = mbar_wait_bounded(&s_bar, phase, nullptr, kWaitLimitNs, a.status);
+    }
+    if (tid == 0) {
+      int ok = mbar_wait_bounded(&s_bar, phase, nullptr, kWaitLimitNs, a.status);
       if (!ok) mbar_wait_bounded(&s_bar, phase, nullptr, kWaitLimitNs, a.status);  // drain
+      s_ok = ok;
     }
-    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncthreads();  // the rows have landed (thread 0 saw the transaction count complete)
+    if (!s_ok) return;
     phase ^= 1u;
-    if (!ok) return;
-    for (int q = lane; q < nr * k; q += 32) {
-      const int i = q / k, j = q - i * k;
+    for (int ij = warp; ij < nr * k; ij += kThreads / 32) {
+      const int i = ij / k, j = ij - i * k;
       const int r = s_rows[r0 + i][j];
-      if (r >= 0) bulk_store(XP + static_cast<size_t>(r) * a.d, s_stage + i * row_bytes, row_bytes);
+      if (r < 0) continue;
+      const uint4* src = reinterpret_cast<const uint4*>(s_stage + i * row_bytes);
+      uint4* dst = reinterpret_cast<uint4*>(XP + static_cast<size_t>(r) * a.d);
+      for (int v = lane; v < nvec; v += 32) dst[v] = src[v];
     }
-    bulk_commit();
-    // The stage is reused by the next round, and must outlive the stores' reads of it
-    // before the CTA exits; the stores then complete on their own.
-    bulk_wait_read_all();
-    __syncwarp();
   }
 }
 
