@@ -83,7 +83,8 @@ Layout layout_of(const moe_config& c) {
   L.stats_partial = c.stats ? take(static_cast<size_t>(kStatsMaxBlocks) * c.E * 8) : 0;
   // Reroute policy (only with it): the router's ranking keys and the list of moved routes.
   L.zkeys = reroute(c) ? take(static_cast<size_t>(c.T) * c.E * 4) : 0;
-  L.rlist = reroute(c) ? take((2 * static_cast<size_t>(c.E) * c.capacity + 1) * 4) : 0;
+  L.rlist = reroute(c) ? take((2 * static_cast<size_t>(c.E) * c.capacity + 1 +
+                                4 * static_cast<size_t>(c.T) * c.k) * 4) : 0;
   L.scratch_end = off;
   L.ids = take(Tk * 4);
   L.gates = take(Tk * 4);

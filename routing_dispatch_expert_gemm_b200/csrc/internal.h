@@ -43,12 +43,13 @@ cudaError_t launch_routing_stats(const moe_config& c, const float* tile_psum,
                                  moe_routing_summary* out, cudaStream_t s);
 
 // Reroute overflow policy on the padded buffer, after the arrival-order pack:
-// assigns the overflowed routes (one CTA, arrival order), rewrites route_row, row_token,
-// the filled-slot counts (offsets[E+2+e]) and the gates of tokens with a moved route,
-// then copies the moved routes' token rows.  list: [2 * E * C + 1] int32 scratch.
+// places the overflowed routes (one CTA, in phases equivalent to the arrival-order walk),
+// rewrites route_row, row_token, the filled-slot counts (offsets[E+2+e]) and the gates of
+// tokens with a moved route, then copies the moved routes' token rows.
+// scratch: [2 * E * C + 1 + 4 * T * k] int32.
 cudaError_t launch_reroute(const moe_config& c, const void* x, const int32_t* ids,
                            const float* zkeys, float* gates, void* x_packed, int32_t* row_token,
-                           int32_t* route_row, int32_t* offsets, int32_t* list,
+                           int32_t* route_row, int32_t* offsets, int32_t* scratch,
                            int32_t* status, cudaStream_t s);
 
 cudaError_t launch_dispatch_hist(const moe_config& c, const int32_t* ids, int32_t* tile_hist,

@@ -5,18 +5,12 @@
 // route is handled by the next-best expert by score, the router's decision overridden).
 //
 // Runs after the arrival-order pack, which has already placed every route that fit and
-// left route_row = -1 on the ones that overflowed.  The reroute is sequential by
-// definition: whether a route finds a free slot depends on every earlier reroute.  One CTA
-// walks the routes in chunks: all threads compact a chunk's overflowed routes (arrival
-// order) and stage their tokens' ranking keys and expert ids in shared memory; then one
-// warp places them one at a time.  In that warp lane l owns experts l, l+32, ..: it keeps
-// their filled-slot counts and the current token's "already held" flags in registers, so a
-// placement is a warp max over an order-preserving integer code of the key (free, not held
-// experts only) and a warp min of the expert index among the maxima -- the router's order
-// and tie rule on the router's own keys -- with no memory round trip on the critical path.
-// The walk stops as soon as no slot is free; the loop keeps all its state in registers and
-// only issues stores.  A second, grid-wide kernel copies each moved route's token row and
-// re-evaluates that token's gates by the gate mode over its final experts.
+// left route_row = -1 on the ones that overflowed.  The reroute is sequential by definition
+// (whether a route finds a free slot depends on every earlier reroute), but because every
+// expert ranks routes by arrival order the result can be built in phases (see
+// reroute_phase_kernel), one CTA, at most E + 1 phases.  A second, grid-wide kernel copies
+// each moved route's token row and re-evaluates that token's gates by the gate mode over its
+// final experts.
 #include <climits>
 
 #include "common.cuh"
@@ -27,20 +21,7 @@ namespace {
 
 constexpr int kThreads = 256;  // copy kernel
 constexpr int kWarps = kThreads / 32;
-constexpr int kAssignThreads = 512;
-constexpr int kAssignWarps = kAssignThreads / 32;
-constexpr int kStageFloats = 16384;  // staged keys per chunk (64 KB)
-constexpr int kStageIds = 16384;     // staged expert ids per chunk (64 KB)
 
-struct AssignArgs {
-  const int32_t* ids;    // [T, k]
-  const float* zkeys;    // [T, E]
-  int32_t* row_token;    // [E * C]
-  int32_t* route_row;    // [T, k]
-  int32_t* offsets;      // segment table; filled-slot counts at offsets[E + 2 + e]
-  int32_t* list;         // [0]: moved routes n, then n (token, row) pairs
-  int T, k, E, C, chunk;
-};
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -52,14 +33,6 @@ __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int s = 16; s >= 1; s >>= 1) v += __shfl_xor_sync(0xffffffffu, v, s);
   return v;
-}
-
-// Order-preserving map of a ranking key (never NaN) to a nonzero unsigned code: a larger
-// key gives a larger code, -0 and +0 the same one, and -inf the smallest (still > 0).
-__device__ __forceinline__ uint32_t key_code(float z) {
-  if (z == 0.f) z = 0.f;
-  const uint32_t u = __float_as_uint(z);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
 // Gates of token t over its final experts (warp-wide; lane j < k writes slot j).  Slot j's
@@ -95,48 +68,106 @@ __device__ void regate(const int32_t* ids, const float* zkeys, const int32_t* ro
   if (lane < k) gates[static_cast<size_t>(t) * k + lane] = g;
 }
 
-// QE: experts per lane of the placing warp, ceil(E / 32) rounded up to a power of two.
-template <int QE>
-__global__ void __launch_bounds__(kAssignThreads, 1) reroute_assign_kernel(AssignArgs a) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  float* s_z = reinterpret_cast<float*>(smem);                                  // [chunk][E]
-  int* s_ids = reinterpret_cast<int*>(smem + static_cast<size_t>(a.chunk) * a.E * 4);  // [chunk][k]
-  __shared__ int s_list[kAssignThreads];
-  __shared__ int s_row[kAssignThreads];  // placed row of each listed route, -1 if none
-  __shared__ int s_mv[kAssignThreads];   // its index in the list of moved routes
-  __shared__ int s_wtot[kAssignWarps];
-  __shared__ int s_n, s_done;
+// ---------------------------------------------------------------------------------
+// Phased placement.  Every expert ranks the overflowed routes by arrival order, so the
+// sequential walk is reproduced exactly in phases: each pending route proposes the expert
+// it would take if the experts full at the phase start were the only full ones (its
+// token's best-ranked expert that it does not hold and that is not full, or the next-best
+// one after the token's earlier routes of the same phase); a scan in arrival order counts
+// each expert's proposals and finds the first route whose expert has run out of slots.
+// Every route before it is placed exactly as the walk would place it.  The phase then
+// restarts at that route with at least one more expert full, so there are at most E + 1
+// phases.  Only routes whose proposal became full (and the later routes of the same
+// token) re-choose.
+// ---------------------------------------------------------------------------------
+constexpr int kPhThreads = 1024;
+constexpr int kPhWarps = kPhThreads / 32;
+
+struct PhaseArgs {
+  const int32_t* ids;      // [T, k]
+  const float* zkeys;      // [T, E]
+  int32_t* row_token;      // [E * C]
+  int32_t* route_row;      // [T, k]
+  int32_t* offsets;        // filled-slot counts at offsets[E + 2 + e]
+  int32_t* list;           // [0]: moved routes n, then (token, row) pairs
+  int32_t* ag_r;           // [T * k] overflowed routes (flat index), arrival order
+  int32_t* ag_c;           // [T * k] proposed / final expert, -1: none
+  int32_t* ag_rank;        // [T * k] rank among the phase's proposals to the same expert
+  int32_t* ag_st;          // [T * k] proposal went stale at the end of the phase
+  int T, k, E, C;
+};
+
+__device__ __forceinline__ bool bit_of(const uint32_t (&w)[8], int e) {
+  uint32_t v = 0;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) v = (q == (e >> 5)) ? w[q] : v;
+  return (v >> (e & 31)) & 1u;
+}
+__device__ __forceinline__ void set_bit(uint32_t (&w)[8], int e) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    if (q == (e >> 5)) w[q] |= 1u << (e & 31);
+}
+
+// The expert route i proposes when the phase starts at `pos` and s_full marks full experts.
+__device__ int propose(const PhaseArgs& a, int i, int pos, const uint32_t* s_full) {
+  const int t = a.ag_r[i] / a.k;
+  uint32_t held[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) held[q] = s_full[q];
+  for (int jj = 0; jj < a.k; ++jj) {
+    const int e = a.ids[static_cast<size_t>(t) * a.k + jj];
+    if (e >= 0 && e < a.E) set_bit(held, e);
+  }
+  int m = 0;  // the token's earlier routes still pending in this phase
+  for (int q = i - 1; q >= 0 && a.ag_r[q] / a.k == t; --q) {
+    if (q >= pos) {
+      ++m;
+    } else {
+      const int cq = a.ag_c[q];
+      if (cq >= 0) set_bit(held, cq);
+    }
+  }
+  const float* zrow = a.zkeys + static_cast<size_t>(t) * a.E;
+  int pick = -1;
+  for (int round = 0; round <= m; ++round) {
+    float bv = -INFINITY;
+    int be = -1;
+    for (int e = 0; e < a.E; ++e) {
+      if (bit_of(held, e)) continue;
+      const float v = zrow[e];
+      if (be < 0 || v > bv) { bv = v; be = e; }  // strict: equal keys keep the lower index
+    }
+    if (be < 0) return -1;
+    set_bit(held, be);
+    pick = be;
+  }
+  return pick;
+}
+
+__global__ void __launch_bounds__(kPhThreads, 1) reroute_phase_kernel(PhaseArgs a) {
+  __shared__ int s_cnt[256], s_carry[256], s_inc[256];
+  __shared__ int s_wc[kPhWarps][256];  // per-warp proposal counts per expert, then bases
+  __shared__ uint32_t s_full[8];
+  __shared__ int s_wtot[kPhWarps];
+  __shared__ int s_n, s_istar, s_moved;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = a.E, k = a.k, C = a.C;
-  // The dependent launch is released only at the end (below): a dependent grid made
-  // resident early would share this CTA's SM while the placing warp runs.
   pdl_wait();  // route_row, counts and the keys come from the router and the pack
 
-  // placing warp's state: counts and held flags of experts lane + 32 q
-  int cnt[QE];
-  bool held[QE];
-  int free_total = 0;
-  if (warp == 0) {
-    int f = 0;
-#pragma unroll
-    for (int q = 0; q < QE; ++q) {
-      const int e = lane + 32 * q;
-      cnt[q] = (e < E) ? a.offsets[E + 2 + e] : C;
-      held[q] = false;
-      f += C - cnt[q];
-    }
-    free_total = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(f)));
-    if (lane == 0) s_done = free_total <= 0 ? 1 : 0;
+  for (int e = tid; e < 256; e += kPhThreads) {
+    s_cnt[e] = (e < E) ? a.offsets[E + 2 + e] : C;
+    s_inc[e] = 0;
   }
+  if (tid == 0) { s_n = 0; s_moved = 0; }
   __syncthreads();
 
+  // 1. overflowed routes, arrival order
   const int total = a.T * k;  // <= INT_MAX / 2 (validated on the host)
-  int cur_t = -1, moved = 0;
-  for (int base = 0; base < total && !s_done; base += a.chunk) {
-    // 1. overflowed routes of this chunk, in arrival order
+  for (int base = 0; base < total; base += kPhThreads) {
     const int r = base + tid;
     bool flag = false;
-    if (tid < a.chunk && r < total) {
+    if (r < total) {
       const int t = r / k, j = r - t * k;
       const int32_t* row = a.ids + static_cast<size_t>(t) * k;
       flag = a.route_row[r] < 0 && route_id_valid(row, j, row[j], E);
@@ -145,87 +176,111 @@ __global__ void __launch_bounds__(kAssignThreads, 1) reroute_assign_kernel(Assig
     if (lane == 0) s_wtot[warp] = __popc(bal);
     __syncthreads();
     int before = 0, n = 0;
-#pragma unroll
-    for (int w = 0; w < kAssignWarps; ++w) {
+    for (int w = 0; w < kPhWarps; ++w) {
       before += (w < warp) ? s_wtot[w] : 0;
       n += s_wtot[w];
     }
-    if (flag) s_list[before + __popc(bal & ((1u << lane) - 1u))] = r;
-    if (tid == 0) s_n = n;
+    if (flag) a.ag_r[s_n + before + __popc(bal & ((1u << lane) - 1u))] = r;
     __syncthreads();
-
-    // 2. stage their tokens' ranking keys and expert ids
-    for (int idx = tid; idx < n * E; idx += kAssignThreads) {
-      const int i = idx / E, e = idx - i * E;
-      s_z[idx] = a.zkeys[static_cast<size_t>(s_list[i] / k) * E + e];
-    }
-    for (int idx = tid; idx < n * k; idx += kAssignThreads) {
-      const int i = idx / k, jj = idx - i * k;
-      s_ids[idx] = a.ids[static_cast<size_t>(s_list[i] / k) * k + jj];
-    }
-    if (tid < n) s_row[tid] = -1;
+    if (tid == 0) s_n += n;
     __syncthreads();
+  }
+  const int n = s_n;
+  if (tid < 8) {
+    uint32_t w = 0;
+    for (int b = 0; b < 32; ++b) {
+      const int e = tid * 32 + b;
+      if (e >= E || s_cnt[e] >= C) w |= 1u << b;
+    }
+    s_full[tid] = w;
+  }
+  __syncthreads();
 
-    // 3. one warp places them in order
-    if (warp == 0) {
-      for (int i = 0; i < n; ++i) {
-        const int rr = s_list[i];
-        const int t = rr / k;
-        if (t != cur_t) {  // a new token: it holds its own top-k experts
-          cur_t = t;
-#pragma unroll
-          for (int q = 0; q < QE; ++q) held[q] = false;
-          for (int jj = 0; jj < k; ++jj) {
-            const int e0 = s_ids[i * k + jj];
-#pragma unroll
-            for (int q = 0; q < QE; ++q) held[q] = held[q] || (e0 == lane + 32 * q);
-          }
+  // 2. first proposals (a token's routes are consecutive, each counts its earlier ones)
+  for (int i = tid; i < n; i += kPhThreads) a.ag_c[i] = propose(a, i, 0, s_full);
+  __syncthreads();
+
+  // 3. phases
+  int pos = 0;
+  while (pos < n) {
+    for (int e = tid; e < 256; e += kPhThreads) s_carry[e] = 0;
+    if (tid == 0) s_istar = n;
+    __syncthreads();
+    for (int base = pos; base < n; base += kPhThreads) {
+      for (int x = tid; x < kPhWarps * 256; x += kPhThreads) (&s_wc[0][0])[x] = 0;
+      __syncthreads();
+      const int i = base + tid;
+      const int c = (i < n) ? a.ag_c[i] : -1;
+      const uint32_t peers = __match_any_sync(0xffffffffu, c);
+      const int wrank = __popc(peers & ((1u << lane) - 1u));
+      if (c >= 0 && wrank == 0) s_wc[warp][c] = __popc(peers);
+      __syncthreads();
+      for (int e = tid; e < E; e += kPhThreads) {  // exclusive prefix over warps
+        int run = s_carry[e];
+        for (int w = 0; w < kPhWarps; ++w) {
+          const int v = s_wc[w][e];
+          s_wc[w][e] = run;
+          run += v;
         }
-        uint32_t best = 0u;
-        unsigned best_e = 0xffffffffu;
-#pragma unroll
-        for (int q = 0; q < QE; ++q) {
-          const int e = lane + 32 * q;
-          if (e < E && !held[q] && cnt[q] < C) {
-            const uint32_t code = key_code(s_z[i * E + e]);
-            if (code > best) { best = code; best_e = static_cast<unsigned>(e); }
-          }
-        }
-        const uint32_t m = __reduce_max_sync(0xffffffffu, best);
-        if (m == 0u) continue;  // no free expert the token does not hold: stays dropped
-        const int es = static_cast<int>(__reduce_min_sync(0xffffffffu, best == m ? best_e : 0xffffffffu));
-        const int owner = es & 31, qs = es >> 5;
-        int slot = 0;
-#pragma unroll
-        for (int q = 0; q < QE; ++q)
-          if (q == qs && lane == owner) { slot = cnt[q]; cnt[q] = slot + 1; held[q] = true; }
-        slot = __shfl_sync(0xffffffffu, slot, owner);
-        if (lane == 0) {  // results go out after the walk, written by the whole CTA
-          s_row[i] = es * C + slot;
-          s_mv[i] = moved;
-        }
-        ++moved;
-        if (--free_total == 0) break;
+        s_carry[e] = run;
       }
-      if (lane == 0) s_done = free_total == 0 ? 1 : 0;
+      __syncthreads();
+      if (c >= 0) {
+        const int rank = s_wc[warp][c] + wrank;
+        a.ag_rank[i] = rank;
+        if (s_cnt[c] + rank >= C) atomicMin(&s_istar, i);
+      }
+      __syncthreads();
+      if (s_istar < n) break;
     }
-    __syncthreads();
-    // 4. write this chunk's placements
-    if (tid < n && s_row[tid] >= 0) {
-      const int rr = s_list[tid], row = s_row[tid], m = s_mv[tid];
-      const int t = rr / k;
-      a.route_row[rr] = row;
+    const int istar = s_istar;
+    // commit the routes before istar
+    for (int i = pos + tid; i < istar; i += kPhThreads) {
+      const int c = a.ag_c[i];
+      if (c < 0) continue;
+      const int r = a.ag_r[i], t = r / k;
+      const int row = c * C + s_cnt[c] + a.ag_rank[i];
+      a.route_row[r] = row;
       a.row_token[row] = t;
+      const int m = atomicAdd(&s_moved, 1);
       a.list[1 + 2 * m] = t;
       a.list[2 + 2 * m] = row;
+      atomicAdd(&s_inc[c], 1);
     }
+    __syncthreads();
+    for (int e = tid; e < E; e += kPhThreads) {
+      s_cnt[e] += s_inc[e];
+      s_inc[e] = 0;
+    }
+    __syncthreads();
+    if (tid < 8) {
+      uint32_t w = 0;
+      for (int b = 0; b < 32; ++b) {
+        const int e = tid * 32 + b;
+        if (e >= E || s_cnt[e] >= C) w |= 1u << b;
+      }
+      s_full[tid] = w;
+    }
+    __syncthreads();
+    pos = istar;
+    if (pos >= n) break;
+    // stale proposals: their expert filled up; later routes of the same token follow them
+    for (int i = pos + tid; i < n; i += kPhThreads) {
+      const int c = a.ag_c[i];
+      a.ag_st[i] = (c >= 0 && ((s_full[c >> 5] >> (c & 31)) & 1u)) ? 1 : 0;
+    }
+    __syncthreads();
+    for (int i = pos + tid; i < n; i += kPhThreads) {
+      const int t = a.ag_r[i] / k;
+      bool redo = a.ag_st[i] != 0;
+      for (int q = i - 1; !redo && q >= pos && a.ag_r[q] / k == t; --q) redo = a.ag_st[q] != 0;
+      if (redo) a.ag_c[i] = propose(a, i, pos, s_full);
+    }
+    __syncthreads();
   }
-  if (warp == 0) {
-#pragma unroll
-    for (int q = 0; q < QE; ++q)
-      if (lane + 32 * q < E) a.offsets[E + 2 + lane + 32 * q] = cnt[q];
-    if (lane == 0) a.list[0] = moved;
-  }
+  for (int e = tid; e < E; e += kPhThreads) a.offsets[E + 2 + e] = s_cnt[e];
+  if (tid == 0) a.list[0] = s_moved;
+  __syncthreads();
   pdl_trigger();
 }
 
@@ -263,34 +318,17 @@ __global__ void __launch_bounds__(kThreads) reroute_copy_kernel(CopyArgs a) {
 
 cudaError_t launch_reroute(const moe_config& c, const void* x, const int32_t* ids,
                            const float* zkeys, float* gates, void* x_packed, int32_t* row_token,
-                           int32_t* route_row, int32_t* offsets, int32_t* list, int32_t* status,
+                           int32_t* route_row, int32_t* offsets, int32_t* scratch, int32_t* status,
                            cudaStream_t s) {
   (void)status;
-  int chunk = kAssignThreads;
-  if (chunk > kStageFloats / c.E) chunk = kStageFloats / c.E;
-  if (chunk > kStageIds / c.k) chunk = kStageIds / c.k;
-  AssignArgs a{ids, zkeys, row_token, route_row, offsets, list, c.T, c.k, c.E, c.capacity, chunk};
-  const size_t smem = static_cast<size_t>(chunk) * (c.E + c.k) * 4;
-  static bool configured = false;
-  if (!configured) {
-    const int lim = (kStageFloats + kStageIds) * 4;
-    cudaFuncSetAttribute(reroute_assign_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
-    cudaFuncSetAttribute(reroute_assign_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
-    cudaFuncSetAttribute(reroute_assign_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
-    cudaFuncSetAttribute(reroute_assign_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
-    configured = true;
-  }
-  cudaError_t e;
-  if (c.E <= 32)
-    e = launch_pdl(reroute_assign_kernel<1>, dim3(1), dim3(kAssignThreads), smem, s, a);
-  else if (c.E <= 64)
-    e = launch_pdl(reroute_assign_kernel<2>, dim3(1), dim3(kAssignThreads), smem, s, a);
-  else if (c.E <= 128)
-    e = launch_pdl(reroute_assign_kernel<4>, dim3(1), dim3(kAssignThreads), smem, s, a);
-  else
-    e = launch_pdl(reroute_assign_kernel<8>, dim3(1), dim3(kAssignThreads), smem, s, a);
+  const size_t slots = static_cast<size_t>(c.E) * c.capacity;
+  const size_t routes = static_cast<size_t>(c.T) * c.k;
+  int32_t* list = scratch;
+  int32_t* ag = scratch + 2 * slots + 1;
+  PhaseArgs a{ids, zkeys, row_token, route_row, offsets, list, ag, ag + routes, ag + 2 * routes,
+              ag + 3 * routes, c.T, c.k, c.E, c.capacity};
+  cudaError_t e = launch_pdl(reroute_phase_kernel, dim3(1), dim3(kPhThreads), 0, s, a);
   if (e != cudaSuccess) return e;
-  long long slots = static_cast<long long>(c.E) * c.capacity;
   int grid = static_cast<int>((slots + kWarps - 1) / kWarps);
   if (grid > 4 * 148) grid = 4 * 148;
   if (grid < 1) grid = 1;
