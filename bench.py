@@ -187,6 +187,25 @@ def source_sha(kernel):
     return h.hexdigest()[:12]
 
 
+# ----------------------------------------------------------------------------- replicas
+
+def max_over_ranks(x, world, device="cpu"):
+    """The largest value of x over all ranks: a job is as slow as its slowest rank.  Every
+    rank must call it at the same point (it is a collective when world > 1)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank_step, world, ms_per_step):
+    """Whole-job throughput: every rank processes units_per_rank_step units per step (weak
+    scaling, independent replicas), and a step takes ms_per_step on the slowest rank."""
+    return world * units_per_rank_step / (ms_per_step / 1e3)
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 
 def blas_threads():
@@ -362,12 +381,9 @@ def run_ours(a):
     unprof = per_step[nprof:] or per_step
     ms_unprofiled = statistics.median(unprof)
     ms_total = sum(per_step)
-    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, world, dev)
     ms_per_step = ms_total / a.steps
-    value = world * wl.T * L / (ms_per_step / 1e3)
+    value = job_throughput(wl.T * L, world, ms_per_step)
     st = N.moe_get_device_status(ws, stream)
     if st != 0:
         raise RuntimeError(f"device status {st} after timing")
@@ -461,12 +477,9 @@ def run_ours(a):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item()) / a.steps
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / a.steps
     nbytes = x.numel() * x.element_size()
-    e2e = {"value": world * wl.T * L / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
+    e2e = {"value": job_throughput(wl.T * L, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
            "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes}
     ok_out = torch.isfinite(y_host.float()).all().item()
     del graphs, g_plain, g_e2e
