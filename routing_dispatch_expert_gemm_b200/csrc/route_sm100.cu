@@ -379,7 +379,7 @@ constexpr int kMaxSmemPerCta = 227 * 1024;
 constexpr int kTokPerCta = kTokens / kCluster;  // 16
 constexpr int kLanesPerTok = 128 / kTokPerCta;  // 8
 
-template <int EN_T, int KMAX>
+template <int EN_T>
 __global__ void __launch_bounds__(kThreads, 1)
     router_cluster_kernel(const __grid_constant__ RouteMaps maps, const RouteParams p) {
   constexpr int V = EN_T / kLanesPerTok;  // logits per lane
@@ -643,29 +643,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 5) tmem_dealloc(tmem_base, p.tmem_cols);
 }
 
-template <int EN_T, int KMAX>
-cudaError_t launch_cluster_kmax(const RouteMaps& maps, const RouteParams& p, int grid, int smem,
-                                cudaStream_t s) {
+template <int EN_T>
+cudaError_t launch_cluster_en(const RouteMaps& maps, const RouteParams& p, int grid, int smem,
+                              cudaStream_t s) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(router_cluster_kernel<EN_T, KMAX>,
+    cudaError_t e = cudaFuncSetAttribute(router_cluster_kernel<EN_T>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmemPerCta);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  return launch_pdl_cluster(router_cluster_kernel<EN_T, KMAX>, dim3(grid), dim3(kThreads), smem,
+  return launch_pdl_cluster(router_cluster_kernel<EN_T>, dim3(grid), dim3(kThreads), smem,
                             kCluster, s, maps, p);
-}
-
-template <int EN_T>
-cudaError_t launch_cluster_en(const RouteMaps& maps, const RouteParams& p, int grid, int smem,
-                              cudaStream_t s) {
-  if (p.k <= 1) return launch_cluster_kmax<EN_T, 1>(maps, p, grid, smem, s);
-  if (p.k <= 2) return launch_cluster_kmax<EN_T, 2>(maps, p, grid, smem, s);
-  if (p.k <= 4) return launch_cluster_kmax<EN_T, 4>(maps, p, grid, smem, s);
-  if (p.k <= 8) return launch_cluster_kmax<EN_T, 8>(maps, p, grid, smem, s);
-  if (p.k <= 16) return launch_cluster_kmax<EN_T, 16>(maps, p, grid, smem, s);
-  return launch_cluster_kmax<EN_T, 32>(maps, p, grid, smem, s);
 }
 
 template <int EN_T, int KMAX>

@@ -25,7 +25,7 @@ def _outputs(cfg, d, dev):
     return dict(x_packed=torch.zeros((rmax, d), dtype=torch.bfloat16, device=dev),
                 row_token=torch.full((rmax,), -7, dtype=torch.int32, device=dev),
                 route_row=torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=dev),
-                offsets=torch.empty(cfg.E + 2, dtype=torch.int32, device=dev),
+                offsets=torch.empty(N.offsets_len(cfg), dtype=torch.int32, device=dev),
                 demand=torch.empty(cfg.E, dtype=torch.int32, device=dev))
 
 
@@ -62,6 +62,25 @@ def test_noalloc_dispatch_matches_workspace_dispatch_twice():
             assert torch.equal(out[key], ref[key]), key
         assert torch.equal(out["row_token"][:R], ref["row_token"][:R])
         assert torch.equal(out["x_packed"][:R].view(torch.int16), ref["x_packed"][:R].view(torch.int16))
+    # the padded [E, C, d] buffer (drop policy): the same comparison over every slot
+    T, E, k, C = 1000, 16, 4, 200
+    cfg = N.make_config(T, d, E, k, 512, capacity=C, layout="padded")
+    ids = I.random_ids(T, E, k, seed=5, skew=1.5).to(dev)
+    x = torch.randn((T, d), generator=torch.Generator().manual_seed(9)).to(torch.bfloat16).to(dev)
+    ref = _outputs(cfg, d, dev)
+    N.moe_dispatch(cfg, x, ids, None, ref["x_packed"], ref["row_token"], ref["route_row"],
+                   ref["offsets"], ref["demand"], N.workspace(cfg))
+    out = _outputs(cfg, d, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    N.moe_dispatch_noalloc(cfg, x, ids, out["x_packed"], out["row_token"], out["route_row"],
+                           out["offsets"], out["demand"], status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for key in ("route_row", "offsets", "demand", "row_token"):
+        assert torch.equal(out[key], ref[key]), key
+    filled = ref["row_token"] >= 0
+    assert int(filled.sum()) == int(ref["offsets"][E + 2:].sum())
+    assert torch.equal(out["x_packed"][filled].view(torch.int16), ref["x_packed"][filled].view(torch.int16))
     # beyond the fixed array: rejected before any launch
     big = N.make_config(1 << 20, 128, 256, 2, 128)
     assert lib.moe_dispatch_noalloc(ctypes.byref(big), 1, 1, 1, 1, 1, 1, 1, None, None) == 2
