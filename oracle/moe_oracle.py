@@ -17,7 +17,7 @@ Sources (web pages, cited by title and section):
   [MoE-S19]   "Mixture-of-Experts: routing and capacity" (Session 19 slides)
   [MoE-AEV]   "Mixture-of-experts routing" (AI Engineering Visualised)
 
-Readings taken where the pages are silent or disagree (each also listed in the design doc):
+Readings taken where the pages are silent or disagree:
   * Three gate modes are kept apart because the pages place the softmax in two places
     (all experts, or only the selected k) and renormalise in one of them.
   * Top-k ranks the logits (softmax is monotone); equal logits go to the lower index.

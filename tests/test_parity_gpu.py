@@ -257,7 +257,7 @@ def _robust_tokens(info, ok, n_near, C):
                                          ("shared64_T16_dropless", 4), ("shared64_T4096_phi1", 6),
                                          ("switch_phi050", 64)])
 def test_full_size_sampled(name, sample):
-    """Full BASELINE-sized layer in the bench's launch configuration; the oracle computes the
+    """Full-size layer in the bench's launch configuration; the oracle computes the
     routing of every token and the output of a seeded sample of tokens."""
     wl = W[name]
     x, (p,) = I.make_inputs(wl, seed=0, device="cuda", layers=1)
