@@ -199,6 +199,76 @@ __global__ void __launch_bounds__(256) combine_bulk_kernel(CombineArgs a) {
   }
 }
 
+// Small k (<= 8): one thread per (token, 16-byte vector) with the token's k rows and gates
+// in registers, loaded straight from global memory (the threads of a warp share a token, so
+// the loads are broadcasts), and the shared-expert and residual rows requested before the
+// gathers since they do not depend on the route table.  Same arithmetic and order as
+// combine_kernel.
+template <typename T, int KMAX>
+__global__ void __launch_bounds__(kThreads) combine_reg_kernel(CombineArgs a) {
+  constexpr int VEC = Vec<T>::N;
+  pdl_trigger();
+  pdl_wait();
+  const int nvec = a.d / VEC;
+  const long long idx = static_cast<long long>(blockIdx.x) * kThreads + threadIdx.x;
+  if (idx >= static_cast<long long>(a.T) * nvec) return;
+  const int t = static_cast<int>(idx / nvec), c = static_cast<int>(idx - static_cast<long long>(t) * nvec);
+  const T* __restrict__ Y = static_cast<const T*>(a.y_packed);
+  const T* __restrict__ R = static_cast<const T*>(a.residual);
+  int rows[KMAX];
+  float g[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    rows[j] = (j < a.k) ? __ldg(a.route_row + static_cast<size_t>(t) * a.k + j) : -1;
+    g[j] = (j < a.k) ? __ldg(a.gates + static_cast<size_t>(t) * a.k + j) : 0.f;
+  }
+  const uint4 rv = (R != nullptr) ? ld_vec(R + static_cast<size_t>(t) * a.d + c * VEC) : make_uint4(0, 0, 0, 0);
+  uint4 sv = make_uint4(0, 0, 0, 0);
+  if (a.has_shared) {
+    const int shared_base = __ldg(a.offsets + a.E);
+    sv = ld_vec(Y + static_cast<size_t>(shared_base + t) * a.d + c * VEC);
+  }
+  uint4 v[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j)
+    v[j] = (rows[j] >= 0) ? ld_vec(Y + static_cast<size_t>(rows[j]) * a.d + c * VEC) : make_uint4(0, 0, 0, 0);
+  float acc[VEC];
+#pragma unroll
+  for (int q = 0; q < VEC; ++q) acc[q] = 0.f;
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    if (rows[j] >= 0) {  // a dropped route contributes nothing
+      float f[VEC];
+      Vec<T>::to_f32(v[j], f);
+#pragma unroll
+      for (int q = 0; q < VEC; ++q) acc[q] = fmaf(g[j], f[q], acc[q]);
+    }
+  }
+  if (a.has_shared) {
+    float f[VEC];
+    Vec<T>::to_f32(sv, f);
+#pragma unroll
+    for (int q = 0; q < VEC; ++q) acc[q] += f[q];
+  }
+  if (R != nullptr) {
+    float f[VEC];
+    Vec<T>::to_f32(rv, f);
+#pragma unroll
+    for (int q = 0; q < VEC; ++q) acc[q] += f[q];
+  }
+  st_vec(static_cast<T*>(a.y) + static_cast<size_t>(t) * a.d + c * VEC, Vec<T>::from_f32(acc));
+}
+
+template <typename T>
+cudaError_t launch_reg(const CombineArgs& a, int nvec, cudaStream_t s) {
+  const long long threads = static_cast<long long>(a.T) * nvec;
+  const int grid = static_cast<int>((threads + kThreads - 1) / kThreads);
+  if (a.k <= 1) return launch_pdl(combine_reg_kernel<T, 1>, dim3(grid), dim3(kThreads), 0, s, a);
+  if (a.k <= 2) return launch_pdl(combine_reg_kernel<T, 2>, dim3(grid), dim3(kThreads), 0, s, a);
+  if (a.k <= 4) return launch_pdl(combine_reg_kernel<T, 4>, dim3(grid), dim3(kThreads), 0, s, a);
+  return launch_pdl(combine_reg_kernel<T, 8>, dim3(grid), dim3(kThreads), 0, s, a);
+}
+
 }  // namespace
 
 cudaError_t launch_combine(const moe_config& c, const void* y_packed, const int32_t* route_row,
@@ -231,6 +301,12 @@ cudaError_t launch_combine(const moe_config& c, const void* y_packed, const int3
     if (c.dtype == MOE_BF16)
       return launch_pdl(combine_bulk_kernel<__nv_bfloat16>, dim3(grid), dim3(threads), bulk_smem, s, a);
     return launch_pdl(combine_bulk_kernel<float>, dim3(grid), dim3(threads), bulk_smem, s, a);
+  }
+  if (c.k <= 8) {
+    CombineArgs a{y_packed, route_row, gates, offsets, c.add_residual ? residual : nullptr,
+                  y, c.T, c.d, c.k, c.E, c.has_shared, 1, nullptr};
+    if (c.dtype == MOE_BF16) return launch_reg<__nv_bfloat16>(a, nvec, s);
+    return launch_reg<float>(a, nvec, s);
   }
   int tpc = kThreads / nvec;
   tpc = tpc < 1 ? 1 : (tpc > kMaxTok ? kMaxTok : tpc);
