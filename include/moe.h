@@ -252,7 +252,7 @@ typedef struct {
   float imbalance;       /* max_e demand_e / mean_e demand_e; 0 when no route is valid       */
   float drop_rate;       /* (T*k - kept) / (T*k)                                             */
   float padding_rate;    /* (E*C - kept) / (E*C) with capacity C > 0; 0 when dropless, C = 0 */
-  int32_t kept;          /* kept routes R = offsets[E]                                       */
+  int32_t kept;          /* kept routes R: offsets[E] (ragged), sum of filled slots (padded) */
   int32_t dropped;       /* T*k - R                                                          */
   int32_t max_demand;    /* max_e demand_e                                                   */
   int32_t busiest_expert;/* lowest e with demand_e = max_demand                              */
@@ -267,6 +267,7 @@ typedef struct {
  *   f_e = demand_e / (T k): routes asking for e before capacity (with top-k each route
  *         counts once, so sum_e f_e = 1 when every id is valid).
  *   P_e = (1/T) sum_t softmax(z_t)_e over all E experts, whatever the gate mode.
+ * With MOE_LAYOUT_PADDED, kept routes are the filled slots (after a reroute, if any).
  * Requires cfg->stats = 1 for the moe_route or moe_forward call that routed on this
  * workspace (its per-tile probability sums are read from `ws`; MOE_ERR_INVALID if
  * cfg->stats is 0).  Sums run in a fixed order (fp32 within a 128-token tile, fp64 across
