@@ -211,3 +211,32 @@ def test_reroute_invariants(name):
     if (gap[over] > 1e-4).all():
         assert r["counts"].tolist() == ref["counts"].tolist()
     assert int(ref["rerouted"].sum()) > 0
+
+
+@pytest.mark.parametrize("overflow", ["drop", "reroute"])
+def test_padded_forward_parity_fp32(overflow):
+    """The fp32 layer (CUDA-core router and grouped GEMMs) through the padded buffer: the
+    GEMMs compute only each expert's filled slots."""
+    wl = W["tiny_fp32"].with_(T=96, E=6, k=2, phi=(1, 1))
+    x_g, (p,) = I.make_inputs(wl, seed=2, device="cuda", layers=1)
+    x, w, b = I.integer_router(wl, seed=8, device="cuda", bias=[3, 2, 0, 0, -1, -2])
+    p = dict(p, w_router=w, logit_bias=b)
+    C = oracle_capacity(wl)
+    cfg = N.make_config(wl.T, wl.d, wl.E, wl.k, wl.d_ff, dtype="f32", gate_mode=wl.gate_mode,
+                        capacity=C, layout="padded", overflow=overflow)
+    ws = N.workspace(cfg)
+    y = torch.empty_like(x)
+    ids = torch.empty((wl.T, wl.k), dtype=torch.int32, device="cuda")
+    gates = torch.empty((wl.T, wl.k), dtype=torch.float32, device="cuda")
+    offsets = torch.empty(N.offsets_len(cfg), dtype=torch.int32, device="cuda")
+    N.moe_forward(cfg, x, p["w_router"], p["logit_bias"], p["w_gate"], p["w_up"], p["w_down"],
+                  None, None, None, y, ids, gates, None, offsets, ws)
+    assert N.moe_get_device_status(ws) == 0
+    y_ref, info = O.moe_layer(x, p, wl.k, wl.gate_mode, C, layout="padded", overflow=overflow)
+    assert np.array_equal(ids.cpu().numpy(), info["ids"])
+    assert offsets.cpu().numpy()[wl.E + 2:].tolist() == info["counts"].tolist()
+    assert int(info["counts"].sum()) < wl.T * wl.k or overflow == "reroute"
+    if overflow == "reroute":
+        assert info["rerouted"].any()
+    assert np.max(np.abs(gates.cpu().numpy() - info["gates"])) <= GATE_ATOL
+    assert_close(y, y_ref, "f32", f"padded fp32/{overflow}")
