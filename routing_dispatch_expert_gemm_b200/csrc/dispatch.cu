@@ -14,7 +14,10 @@
 // The first term is an exclusive prefix over the per-128-token-tile histogram; every CTA
 // computes the prefix it needs directly from the histogram (ceil(T/128) x E entries), so
 // no separate scan launch and no inter-CTA waiting is needed.  Pack CTAs cover 8-token
-// sub-tiles of a histogram tile, so the copy work spreads over many SMs.
+// sub-tiles of a histogram tile, so the copy work spreads over many SMs.  A CTA starts the
+// bulk loads of its token rows first (they do not depend on the routing), works out the
+// positions meanwhile, then all its warps write each row to its kept routes' rows.  With
+// the padded [E, C, d] buffer expert e's rows start at e*C and empty slots are marked -1.
 #include "common.cuh"
 #include "internal.h"
 

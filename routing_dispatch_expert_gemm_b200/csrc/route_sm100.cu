@@ -9,14 +9,18 @@
 // "MoE Inference Visualized", The Router (the top-1 weight is the softmax probability);
 // "Mixture-of-experts routing", The gate (softmax over only the top-k).
 //
-// One CTA per 128 tokens.  The logit contraction [128 x d] x [d x E] runs as tcgen05.mma
-// with M = 128 tokens and N = E rounded up to 16 experts, fp32 accumulation in tensor
-// memory; x streams through a deep TMA ring (the router-weight tile per stage is small, so
-// up to 12 stages fit).  The epilogue gives each thread one token (one TMEM lane): it reads
-// the token's E logits in 16-column chunks, keeps a sorted top-KMAX list in registers
-// (insertion in expert order, so an equal logit never displaces an earlier expert), then
-// forms the gates and adds the token's experts to the tile histogram.  For E <= 64 the
-// token's logits stay in registers and top-k is a tournament (see topk_tournament).
+// The logit contraction [128 tokens x d] x [d x E] runs as tcgen05.mma with M = 128 tokens
+// and N = E rounded up to 16 experts, fp32 accumulation in tensor memory, x streaming
+// through a TMA ring.  Two kernels:
+//  * router_cluster_kernel (E <= 64, d >= 512): a cluster of 8 CTAs shares a 128-token tile,
+//    each contracting 1/8 of d; the partial logits are summed in distributed shared memory
+//    in rank order, and top-k is a rank count with 8 lanes per token (see the kernel).
+//  * router_tc_kernel (otherwise): one CTA per tile; each thread owns one token (one TMEM
+//    lane).  For E <= 64 its logits stay in registers and top-k is a tournament (see
+//    topk_tournament); above that it reads 16-column chunks into a sorted top-KMAX list
+//    (insertion in expert order, so an equal logit never displaces an earlier expert).
+// Both form the gates and the tile's expert histogram, and optionally the per-tile sums of
+// the full softmax (routing statistics) and the ranking keys (reroute policy).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
