@@ -1,9 +1,10 @@
 """Routing statistics on the GPU (moe_routing_stats) against the fp64 oracle.
 
-f, kept/dropped counts, imbalance, drop and padding rates are functions of the expert ids;
-they are compared with the oracle evaluated on the ids the GPU chose (those ids are checked
-against the oracle's own, near ties excluded, here and in the route parity tests): f bit-exact
-(the same correctly rounded quotient), the counts exact, the rates to fp32 rounding.
+f, kept/dropped counts, imbalance, drop and padding rates are functions of the expert ids.
+The oracle routes on its own; where the GPU chose the same expert set for every token (the
+usual case) they are compared exactly: f bit-exact (the same correctly rounded quotient), the
+counts exact, the rates to fp32 rounding.  Where near-tie tokens (logits within 1e-4) chose a
+different set, each such token moves at most k routes, which bounds the differences.
 P (mean full-softmax probability) is compared with the oracle's fp64 softmax of the same
 stored inputs within P_RTOL: the kernel's logits carry fp32 accumulation error (|dz| well
 under 1e-5 for these shapes), a probability moves by p * |dz| to first order, and the fp32
@@ -49,6 +50,41 @@ CASES = {
 }
 
 
+def _check_against_oracle(wl, x, p, C, ids, f, P, s, demand):
+    """Compare the GPU's statistics with the oracle's, computed from the oracle's own routing."""
+    ref_ids, _, z = O.route(x, p["w_router"], p["logit_bias"], wl.k, wl.gate_mode)
+    bad, _, _ = ids_agree(ids, ref_ids, O.topk_margin(z, wl.k), z, wl.k)
+    assert len(bad) == 0
+    ref = O.routing_stats(x, p["w_router"], p["logit_bias"], wl.k, C, alpha=ALPHA)
+    dem_ref = O.dispatch(ref_ids, wl.E, C)["demand"]
+    # P is the full softmax, whatever experts were chosen
+    Pg = P.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(Pg - ref["P"]) <= P_RTOL * ref["P"] + 1e-9), np.max(np.abs(Pg - ref["P"]))
+    g = ids.cpu().numpy().astype(np.int64)
+    moved = int((np.sort(g, axis=1) != np.sort(ref_ids, axis=1)).any(axis=1).sum())
+    dem = demand.cpu().numpy().astype(np.int64)
+    Tk = wl.T * wl.k
+    if moved == 0:
+        assert dem.tolist() == dem_ref.tolist()
+        if f is not None:
+            assert np.array_equal(f.cpu().numpy(), ref["f"].astype(np.float32))
+        assert abs(s["aux_loss"] - ref["aux"]) <= P_RTOL * ref["aux"] + 1e-9
+        assert s["kept"] == ref["kept"] and s["dropped"] == Tk - ref["kept"]
+        assert s["imbalance"] == np.float32(ref["imbalance"])
+        assert s["drop_rate"] == np.float32(ref["drop_rate"])
+        assert s["padding_rate"] == np.float32(ref["padding_rate"])
+    else:  # each differing token shifts at most k routes between experts
+        assert np.abs(dem - dem_ref).sum() <= 2 * wl.k * moved
+        assert abs(s["kept"] - ref["kept"]) <= 2 * wl.k * moved
+        bound = ALPHA * wl.E * float(np.sum(np.abs(dem - dem_ref) / Tk * ref["P"]))
+        assert abs(s["aux_loss"] - ref["aux"]) <= P_RTOL * ref["aux"] + bound + 1e-9
+    # the summary is consistent with the GPU's own counts in every case
+    assert s["max_demand"] == dem.max() and s["busiest_expert"] == int(np.argmax(dem))
+    assert s["dropped"] == Tk - s["kept"]
+    if f is not None:
+        assert np.array_equal(f.cpu().numpy(), (dem / Tk).astype(np.float32))
+
+
 def _route_dispatch_stats(wl, cfg, x, p, ws):
     dev = x.device
     T, k, E = wl.T, wl.k, wl.E
@@ -78,24 +114,7 @@ def test_routing_stats_parity(name):
     ws = N.workspace(cfg)
     ids, demand, _, f, P, summ = _route_dispatch_stats(wl, cfg, x, p, ws)
     s = N.summary_dict(summ)
-
-    C = oracle_capacity(wl)
-    ids_np = ids.cpu().numpy().astype(np.int64)
-    ref_ids, _, z = O.route(x, p["w_router"], p["logit_bias"], wl.k, wl.gate_mode)
-    bad, _, _ = ids_agree(ids, ref_ids, O.topk_margin(z, wl.k), z, wl.k)
-    assert len(bad) == 0
-    ref = O.routing_stats(x, p["w_router"], p["logit_bias"], wl.k, C, alpha=ALPHA, ids=ids_np)
-
-    assert np.array_equal(f.cpu().numpy(), ref["f"].astype(np.float32))
-    Pg = P.cpu().numpy().astype(np.float64)
-    assert np.all(np.abs(Pg - ref["P"]) <= P_RTOL * ref["P"] + 1e-9), np.max(np.abs(Pg - ref["P"]))
-    assert abs(s["aux_loss"] - ref["aux"]) <= P_RTOL * ref["aux"] + 1e-9
-    dem = demand.cpu().numpy()
-    assert s["kept"] == ref["kept"] and s["dropped"] == wl.T * wl.k - ref["kept"]
-    assert s["max_demand"] == dem.max() and s["busiest_expert"] == int(np.argmax(dem))
-    assert s["imbalance"] == np.float32(ref["imbalance"])
-    assert s["drop_rate"] == np.float32(ref["drop_rate"])
-    assert s["padding_rate"] == np.float32(ref["padding_rate"])
+    _check_against_oracle(wl, x, p, oracle_capacity(wl), ids, f, P, s, demand)
 
 
 def test_routing_stats_repeatable():
@@ -138,9 +157,4 @@ def test_forward_with_stats():
     assert N.moe_get_device_status(ws) == 0
     assert torch.equal(f, f_ref) and torch.equal(summ, summ_ref)
     s = N.summary_dict(summ)
-    C = oracle_capacity(wl)
-    ref = O.routing_stats(x, p["w_router"], p["logit_bias"], wl.k, C, alpha=ALPHA,
-                          ids=plain["ids"].cpu().numpy().astype(np.int64))
-    assert s["kept"] == ref["kept"]
-    Pg = P.cpu().numpy().astype(np.float64)
-    assert np.all(np.abs(Pg - ref["P"]) <= P_RTOL * ref["P"] + 1e-9)
+    _check_against_oracle(wl, x, p, oracle_capacity(wl), plain["ids"], f, P, s, plain["demand"])
