@@ -37,10 +37,7 @@ namespace {
 constexpr int kTokens = 128;           // tokens per CTA = MMA M = TMEM lanes
 constexpr int BK = 64;                 // 128-byte swizzle rows of bf16
 constexpr int kThreads = 192;          // warps 0-3 epilogue, 4 TMA producer, 5 MMA
-#ifndef MOE_ROUTER_MAX_STAGES
-#define MOE_ROUTER_MAX_STAGES 12
-#endif
-constexpr int kMaxStages = MOE_ROUTER_MAX_STAGES;
+constexpr int kMaxStages = 12;         // deepest TMA ring (the router-weight tile is small)
 constexpr int A_BYTES = kTokens * BK * 2;
 constexpr int kRingBudget = 192 * 1024;
 
