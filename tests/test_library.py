@@ -158,3 +158,38 @@ def test_layout_and_overflow_validation(native):
     assert lib.moe_dispatch_noalloc(ctypes.byref(native.make_config(
         8, 128, 4, 2, 128, layout="padded")), fake, fake, fake, fake, fake, fake, fake, None,
         None) == 1
+
+
+def test_config_sweep_validation_and_sizes(native):
+    """Random configs: valid ones get a 256-byte-aligned workspace and the documented row
+    bound; each optional feature only adds scratch; invalid combinations are rejected."""
+    import random
+    rng = random.Random(0)
+    for _ in range(400):
+        E = rng.choice([1, 2, 4, 8, 32, 64, 200, 256])
+        k = rng.randint(1, min(E, 32))
+        T = rng.choice([1, 7, 128, 129, 1000, 4096])
+        dtype = rng.choice(["bf16", "f32"])
+        d = rng.choice([128, 256, 1024]) if dtype == "bf16" else rng.choice([4, 64, 100])
+        F = rng.choice([128, 512]) if dtype == "bf16" else rng.choice([4, 128])
+        cap = rng.choice([-1, 0, 1, 17, T * k])
+        layout = rng.choice(["ragged", "padded"])
+        overflow = rng.choice(["drop", "reroute"])
+        cfg = native.make_config(T, d, E, k, F, dtype=dtype, capacity=cap, layout=layout,
+                                 overflow=overflow, has_shared=rng.random() < 0.3,
+                                 add_residual=rng.random() < 0.5, stats=rng.random() < 0.5)
+        ws = native.moe_workspace_bytes(cfg)
+        if layout == "padded" and cap < 0:
+            assert ws == 0                       # the padded buffer needs C
+            continue
+        if overflow == "reroute" and layout != "padded":
+            assert ws == 0                       # reroute fills the padded buffer's slots
+            continue
+        assert ws > 0 and ws % 256 == 0, (cfg, ws)
+        rows = native.moe_max_rows(cfg)
+        if layout == "padded":
+            assert rows == max(E * cap, 1)
+        else:
+            assert rows == max(min(T * k, E * cap) if cap >= 0 else T * k, 1)
+        base = native.make_config(T, d, E, k, F, dtype=dtype, capacity=cap, layout=layout)
+        assert native.moe_workspace_bytes(base) <= ws
