@@ -57,6 +57,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the workload's layer count (a stack of fewer layers)")
+    ap.add_argument("--stats", action="store_true",
+                    help="also gather routing statistics: the router's per-tile sums and one "
+                         "moe_routing_stats call per layer")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="launch through the library call by call instead of replaying a CUDA graph")
     a = ap.parse_args()
@@ -284,8 +287,9 @@ def run_ours(a):
     cap = -1 if wl.phi is None else N.moe_capacity(wl.T, wl.k, wl.E, *wl.phi)
     cfg = N.make_config(wl.T, wl.d, wl.E, wl.k, wl.d_ff, dtype=wl.dtype, gate_mode=wl.gate_mode,
                         capacity=cap, has_shared=wl.has_shared, add_residual=wl.add_residual,
-                        layout=wl.layout, overflow=wl.overflow)
+                        layout=wl.layout, overflow=wl.overflow, stats=a.stats)
     ws = N.workspace(cfg, dev)
+    summ = torch.zeros((L, 32), dtype=torch.uint8, device=dev)
     ybuf = [torch.empty_like(x), torch.empty_like(x)]
     demand = torch.zeros((L, wl.E), dtype=torch.int32, device=dev)
     offsets = torch.zeros((L, N.offsets_len(cfg)), dtype=torch.int32, device=dev)
@@ -303,6 +307,8 @@ def run_ours(a):
                 N.moe_forward(*args, ws, st_)
             else:
                 N.moe_forward_profiled(*args, evs[l], ws, st_)
+            if a.stats:
+                N.moe_routing_stats(cfg, demand[l], offsets[l], 1e-2, None, None, summ[l], ws, st_)
             h = y
         return h
 
@@ -512,12 +518,14 @@ def run_ours(a):
                    "d_ff": wl.d_ff, "layers": L, "gate_mode": wl.gate_mode,
                    "capacity": cap, "shared_expert": wl.has_shared,
                    "residual": wl.add_residual, "layout": wl.layout, "overflow": wl.overflow,
+                   "routing_stats": a.stats,
                    "parallelism": f"replicas{world}",
                    "cuda_graph": a.graph,
                    "l2": ("flushed between steps" if flush is not None else
                           f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB of weights per step)")},
         "roofline": roofline, "kernels": breakdown, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": a.steps * L * (7 if wl.overflow == "reroute" else 5), "clocks": clk,
+        "gpu_launches": a.steps * L * ((7 if wl.overflow == "reroute" else 5) + int(a.stats)),
+        "clocks": clk,
         "routes_per_step": int(dem.sum()), "output_finite": bool(ok_out),
     }
     print(json.dumps(out), flush=True)
