@@ -230,8 +230,11 @@ moe_status moe_debug_bounded_wait(void* ws, int64_t limit_ns, moe_stream_t strea
  *   process exits).  Configurations whose histogram, ceil(T / tile) * E entries with the
  *   token tile of moe_dispatch, exceeds 16384 entries are rejected with
  *   MOE_ERR_UNSUPPORTED; nothing is launched then.
- *   Set-up: the first call on a device looks up the array's device address (once per
- *   device, with that device current); make that first call before any stream capture.
+ *   Set-up: every call looks up the array's device address in the current device's
+ *   context (a host-side query that enqueues no work), so the address stays right after
+ *   cudaDeviceReset or under another context on the same device.  The first call on a
+ *   device may load the library's device code for that context: make that first call
+ *   before any stream capture.
  *   Sharing: every call on a device uses the same array and it keeps the last call's
  *   contents; nothing in it needs to start at zero because each call rewrites the entries
  *   it reads.  Calls that overlap on the GPU (other streams, other host threads) race on

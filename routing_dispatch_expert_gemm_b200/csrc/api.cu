@@ -10,13 +10,11 @@
 
 using namespace moe;
 
-namespace {
+namespace moe {
 
-constexpr int32_t kAbiVersion = 3;
-
-size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
-
-moe_status validate(const moe_config* c) {
+// Host-side checks shared by every entry point that takes a config (declared in
+// internal.h).
+moe_status validate_config(const moe_config* c) {
   if (c == nullptr) return MOE_ERR_INVALID;
   if (c->T < 1 || c->d < 1 || c->E < 1 || c->k < 1 || c->d_ff < 1) return MOE_ERR_INVALID;
   if (c->k > c->E) return MOE_ERR_INVALID;
@@ -43,6 +41,16 @@ moe_status validate(const moe_config* c) {
   }
   return MOE_OK;
 }
+
+}  // namespace moe
+
+namespace {
+
+moe_status validate(const moe_config* c) { return validate_config(c); }
+
+constexpr int32_t kAbiVersion = 3;
+
+size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 int64_t max_rows(const moe_config& c) {
   if (c.layout == MOE_LAYOUT_PADDED)

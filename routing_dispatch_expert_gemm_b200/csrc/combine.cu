@@ -288,16 +288,19 @@ cudaError_t launch_combine(const moe_config& c, const void* y_packed, const int3
     CombineArgs a{y_packed, route_row, gates, offsets, c.add_residual ? residual : nullptr,
                   y, c.T, c.d, c.k, c.E, c.has_shared, tpc, nullptr};
     const int grid = (c.T + tpc - 1) / tpc;
-    static bool configured = false;
-    if (!configured) {
+    static DeviceOnce once;
+    cudaError_t e = once.run([] {
       prefer_max_shared(combine_bulk_kernel<__nv_bfloat16>);
       prefer_max_shared(combine_bulk_kernel<float>);
-      cudaFuncSetAttribute(combine_bulk_kernel<__nv_bfloat16>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kBulkSmemMax));
-      cudaFuncSetAttribute(combine_bulk_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kBulkSmemMax));
-      configured = true;
-    }
+      cudaError_t r = cudaFuncSetAttribute(combine_bulk_kernel<__nv_bfloat16>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(kBulkSmemMax));
+      if (r != cudaSuccess) return r;
+      return cudaFuncSetAttribute(combine_bulk_kernel<float>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(kBulkSmemMax));
+    });
+    if (e != cudaSuccess) return e;
     if (c.dtype == MOE_BF16)
       return launch_pdl(combine_bulk_kernel<__nv_bfloat16>, dim3(grid), dim3(threads), bulk_smem, s, a);
     return launch_pdl(combine_bulk_kernel<float>, dim3(grid), dim3(threads), bulk_smem, s, a);
@@ -313,12 +316,12 @@ cudaError_t launch_combine(const moe_config& c, const void* y_packed, const int3
   CombineArgs a{y_packed, route_row, gates, offsets, c.add_residual ? residual : nullptr,
                 y, c.T, c.d, c.k, c.E, c.has_shared, tpc, nullptr};
   const int grid = (c.T + tpc - 1) / tpc;
-  static bool configured = false;
-  if (!configured) {
+  static DeviceOnce once;
+  cudaError_t e = once.run([] {
     prefer_max_shared(combine_kernel<__nv_bfloat16>);
-    prefer_max_shared(combine_kernel<float>);
-    configured = true;
-  }
+    return prefer_max_shared(combine_kernel<float>);
+  });
+  if (e != cudaSuccess) return e;
   if (c.dtype == MOE_BF16)
     return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(kThreads), 0, s, a);
   return launch_pdl(combine_kernel<float>, dim3(grid), dim3(kThreads), 0, s, a);

@@ -6,6 +6,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "moe.h"
 
 namespace moe {
@@ -97,6 +100,34 @@ inline cudaError_t prefer_max_shared(K kernel) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                               cudaSharedmemCarveoutMaxShared);
 }
+
+// ---------------------------------------------------------------------------------
+// One-time host set-up per device.  Kernel attributes (dynamic shared-memory limit,
+// carveout) apply to the current device only, so each launcher keeps one DeviceOnce and
+// runs its set-up the first time it launches on each device.  Thread-safe; a set-up that
+// fails is retried on the next call.
+// ---------------------------------------------------------------------------------
+class DeviceOnce {
+ public:
+  template <typename F>
+  cudaError_t run(F&& setup) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (done_[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    std::lock_guard<std::mutex> lock(mu_);
+    if (done_[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+    e = setup();
+    if (e == cudaSuccess) done_[dev].store(1, std::memory_order_release);
+    return e;
+  }
+
+ private:
+  static constexpr int kMaxDevices = 64;
+  std::atomic<int> done_[kMaxDevices] = {};
+  std::mutex mu_;
+};
 
 // ---------------------------------------------------------------------------------
 // Programmatic dependent launch.  Every kernel of the forward is launched so that it may

@@ -250,11 +250,9 @@ cudaError_t launch_dispatch_hist(const moe_config& c, const int32_t* ids, int32_
                                  int32_t* status, cudaStream_t s) {
   const int tt = tok_tile_for(c.T, c.E);
   const int grid = (c.T + tt - 1) / tt;
-  static bool configured = false;
-  if (!configured) {
-    prefer_max_shared(hist_kernel);
-    configured = true;
-  }
+  static DeviceOnce once;
+  cudaError_t e = once.run([] { return prefer_max_shared(hist_kernel); });
+  if (e != cudaSuccess) return e;
   return launch_pdl(hist_kernel, dim3(grid), dim3(kThreads), 0, s, ids, c.T, c.k, c.E, tt,
                     tile_hist, status);
 }
@@ -271,16 +269,18 @@ cudaError_t launch_dispatch_scatter(const moe_config& c, const void* x, const in
                 c.capacity, c.has_shared, round, c.layout == MOE_LAYOUT_PADDED ? 1 : 0, x_packed,
                 row_token, route_row, offsets, demand, status};
   const size_t smem = static_cast<size_t>(round) * row_bytes;
-  static bool configured = false;
-  if (!configured) {
+  static DeviceOnce once;
+  cudaError_t e = once.run([] {
     prefer_max_shared(scatter_kernel<__nv_bfloat16>);
     prefer_max_shared(scatter_kernel<float>);
-    cudaFuncSetAttribute(scatter_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(kStageBudget));
-    cudaFuncSetAttribute(scatter_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(kStageBudget));
-    configured = true;
-  }
+    cudaError_t r = cudaFuncSetAttribute(scatter_kernel<__nv_bfloat16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kStageBudget));
+    if (r != cudaSuccess) return r;
+    return cudaFuncSetAttribute(scatter_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(kStageBudget));
+  });
+  if (e != cudaSuccess) return e;
   if (c.dtype == MOE_BF16)
     return launch_pdl(scatter_kernel<__nv_bfloat16>, dim3(grid), dim3(kThreads), smem, s, a);
   return launch_pdl(scatter_kernel<float>, dim3(grid), dim3(kThreads), smem, s, a);

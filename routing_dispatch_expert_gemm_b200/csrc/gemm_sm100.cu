@@ -366,27 +366,27 @@ bool encode_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows) {
   return encode_2d_box(m, ptr, cols, rows, kBoxRows);
 }
 
+// SMs of the current device (a cheap host query, made per launch so that every device
+// gets its own count).
 int sm_count() {
-  static int n = [] {
-    int dev = 0, v = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    return v > 0 ? v : 148;
-  }();
-  return n;
+  int dev = 0, v = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+    return 148;
+  return v;
 }
 
 template <int MODE, int BN>
 cudaError_t launch_gemm(const Maps& maps, const Params& p, long long tiles_bound, cudaStream_t s) {
   using C = Cfg<MODE, BN>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, BN>,
+  static DeviceOnce once;
+  cudaError_t e = once.run([] {
+    cudaError_t r = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, BN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    prefer_max_shared(grouped_gemm_kernel<MODE, BN>);
-    configured = true;
-  }
+    if (r != cudaSuccess) return r;
+    return prefer_max_shared(grouped_gemm_kernel<MODE, BN>);
+  });
+  if (e != cudaSuccess) return e;
   const int grid = static_cast<int>(tiles_bound < sm_count() ? (tiles_bound > 0 ? tiles_bound : 1)
                                                              : sm_count());
   return launch_pdl(grouped_gemm_kernel<MODE, BN>, dim3(grid), dim3(kThreads), C::SMEM, s, maps, p);

@@ -8,6 +8,10 @@
 
 namespace moe {
 
+// Host-side validation of a config: MOE_OK, MOE_ERR_INVALID or MOE_ERR_UNSUPPORTED (the
+// same checks every entry point that takes a config applies before any launch).
+moe_status validate_config(const moe_config* c);
+
 // Token tile of the expert histogram that connects routing and packing: 128 tokens, the
 // router's CTA tile (one TMEM lane per token).  The histogram is num_tiles x E int32.
 constexpr int kHistTile = 128;

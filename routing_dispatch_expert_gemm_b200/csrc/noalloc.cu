@@ -8,8 +8,6 @@
 // the device or take a global lock).  This variant therefore keeps its only scratch, the
 // per-token-tile expert histogram, in a fixed array in the library's own device memory
 // and takes no workspace argument.  The caller still passes inputs and outputs.
-#include <mutex>
-
 #include "common.cuh"
 #include "internal.h"
 
@@ -21,26 +19,17 @@ namespace {
 constexpr int kNoAllocHistEntries = 16384;  // 64 KiB
 static __device__ __align__(256) int32_t g_noalloc_hist[kNoAllocHistEntries];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-int32_t* g_hist_ptr[kMaxDevices] = {};
-
-// Device address of g_noalloc_hist on the current device.  In host code the symbol
-// names a host-side stand-in, not device memory, so the address must be looked up, once
-// per device, with that device current.
+// Device address of g_noalloc_hist in the current device's context.  In host code the
+// symbol names a host-side stand-in, not device memory, so the address is looked up with
+// the device current.  The lookup is a host-side query that enqueues no work; it is made
+// on every call rather than cached, because the address belongs to the context that
+// loaded the module: after cudaDeviceReset, or under another context on the same device,
+// an address kept from an earlier call would point at memory that is no longer ours.
 cudaError_t hist_address(int32_t** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_hist);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (g_hist_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_hist);
-    if (e != cudaSuccess) return e;
-    g_hist_ptr[dev] = static_cast<int32_t*>(p);
-  }
-  *out = g_hist_ptr[dev];
+  *out = static_cast<int32_t*>(p);
   return cudaSuccess;
 }
 
@@ -54,23 +43,11 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_config* cfg, const void* x,
                                            int32_t* row_token, int32_t* route_row,
                                            int32_t* offsets, int32_t* demand, int32_t* status,
                                            moe_stream_t stream) {
-  // Same argument checks as moe_dispatch (validation lives in api.cu; repeated here in
-  // short form so this file stays independent of the workspace layout).
-  if (cfg == nullptr || cfg->T < 1 || cfg->d < 1 || cfg->E < 1 || cfg->k < 1 || cfg->k > cfg->E ||
-      (cfg->dtype != MOE_F32 && cfg->dtype != MOE_BF16))
-    return MOE_ERR_INVALID;
-  if ((cfg->layout != MOE_LAYOUT_RAGGED && cfg->layout != MOE_LAYOUT_PADDED) ||
-      (cfg->overflow != MOE_OVERFLOW_DROP && cfg->overflow != MOE_OVERFLOW_REROUTE) ||
-      (cfg->layout == MOE_LAYOUT_PADDED && cfg->capacity < 0))
-    return MOE_ERR_INVALID;
+  // The checks every entry point applies, then the two limits of this one.
+  const moe_status v = validate_config(cfg);
+  if (v != MOE_OK) return v;
   // The reroute policy ranks with the router's logits, which live in a workspace.
   if (cfg->overflow == MOE_OVERFLOW_REROUTE) return MOE_ERR_UNSUPPORTED;
-  if (cfg->E > 256 || cfg->k > 32 || cfg->T > (1 << 24)) return MOE_ERR_UNSUPPORTED;
-  if (static_cast<long long>(cfg->T) * cfg->k > (1 << 30) ||
-      (cfg->layout == MOE_LAYOUT_PADDED && static_cast<long long>(cfg->E) * cfg->capacity > (1 << 30)))
-    return MOE_ERR_UNSUPPORTED;
-  if ((cfg->dtype == MOE_BF16 && cfg->d % 128 != 0) || (cfg->dtype == MOE_F32 && cfg->d % 4 != 0))
-    return MOE_ERR_UNSUPPORTED;
   if (!x || !ids || !x_packed || !row_token || !route_row || !offsets || !demand)
     return MOE_ERR_INVALID;
   // The histogram must fit the fixed array.

@@ -249,13 +249,12 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(RouterArgs a) {
 template <typename Tin, int EP>
 cudaError_t launch_ep(const RouterArgs& a, int grid, cudaStream_t s) {
   const int smem = EP * a.dc * static_cast<int>(sizeof(Tin));
-  static bool configured = false;  // attribute set once per instantiation
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(router_kernel<Tin, EP>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kWChunkBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static DeviceOnce once;  // attribute set once per instantiation and device
+  cudaError_t e = once.run([] {
+    return cudaFuncSetAttribute(router_kernel<Tin, EP>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, kWChunkBytes);
+  });
+  if (e != cudaSuccess) return e;
   return launch_pdl(router_kernel<Tin, EP>, dim3(grid), dim3(kThreads), smem, s, a);
 }
 

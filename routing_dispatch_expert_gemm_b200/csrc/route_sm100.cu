@@ -647,13 +647,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int EN_T>
 cudaError_t launch_cluster_en(const RouteMaps& maps, const RouteParams& p, int grid, int smem,
                               cudaStream_t s) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(router_cluster_kernel<EN_T>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmemPerCta);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static DeviceOnce once;
+  cudaError_t e = once.run([] {
+    return cudaFuncSetAttribute(router_cluster_kernel<EN_T>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmemPerCta);
+  });
+  if (e != cudaSuccess) return e;
   return launch_pdl_cluster(router_cluster_kernel<EN_T>, dim3(grid), dim3(kThreads), smem,
                             kCluster, s, maps, p);
 }
@@ -661,15 +660,15 @@ cudaError_t launch_cluster_en(const RouteMaps& maps, const RouteParams& p, int g
 template <int EN_T, int KMAX>
 cudaError_t launch_kmax(const RouteMaps& maps, const RouteParams& p, int grid, int smem,
                         cudaStream_t s) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<EN_T, KMAX>,
+  static DeviceOnce once;
+  cudaError_t e = once.run([] {
+    cudaError_t r = cudaFuncSetAttribute(router_tc_kernel<EN_T, KMAX>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          1024 + kRingBudget + 8192);
-    if (e != cudaSuccess) return e;
-    prefer_max_shared(router_tc_kernel<EN_T, KMAX>);
-    configured = true;
-  }
+    if (r != cudaSuccess) return r;
+    return prefer_max_shared(router_tc_kernel<EN_T, KMAX>);
+  });
+  if (e != cudaSuccess) return e;
   return launch_pdl(router_tc_kernel<EN_T, KMAX>, dim3(grid), dim3(kThreads), smem, s, maps, p);
 }
 
