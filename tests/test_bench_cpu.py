@@ -59,3 +59,29 @@ def test_committed_granite_traffic_is_current_or_absent():
     reported against a kernel it was not measured on)."""
     t = bench.traffic_from_profiles("gemm_gate_up", "granite24")
     assert t is None or 50e6 < t < 120e6
+
+
+def test_default_workload_is_the_largest_single_gpu_configuration():
+    """With no flags the headline is the 64+1 layer at T=4096 (the largest configuration that
+    fits one GPU), and the other configurations follow under 'workloads'."""
+    a = bench.parse_args([])
+    wl = I.WORKLOADS[a.workload]
+    assert (wl.T, wl.d, wl.E, wl.k, wl.d_ff, wl.has_shared) == (4096, 4096, 64, 2, 32768, True)
+    sizes = {n: w.T * w.d * w.d_ff * (w.E + int(w.has_shared)) for n, w in I.WORKLOADS.items()}
+    assert sizes[a.workload] == max(sizes.values())
+    assert a.workload not in a.also
+    for name in ("granite24", "mixtral_prefill", "mixtral_decode", "shared64_T16_dropless"):
+        assert name in a.also
+    assert a.warmup >= 3
+    assert bench.parse_args(["--also", "none"]).also == []
+    assert bench.parse_args(["--workload", "granite24", "--also", "granite24,mixtral_decode"]).also \
+        == ["mixtral_decode"]
+
+
+def test_oracle_sample_is_bounded_for_large_layers():
+    """The CPU baseline computes every token of small layers and a few tokens of the layers
+    whose experts are large (each touched expert costs 3 d F fp64 values)."""
+    assert bench.oracle_tokens(I.WORKLOADS["tiny_fp32"]) is None
+    assert bench.oracle_tokens(I.WORKLOADS["granite24"]) is None
+    assert bench.oracle_tokens(I.WORKLOADS["mixtral_prefill"]) == 32
+    assert bench.oracle_tokens(I.WORKLOADS["shared64_T4096_dropless"]) == 4
