@@ -48,8 +48,10 @@ SPEC_PEAKS = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}
 KERNELS = ["route", "pack", "gemm_gate_up", "gemm_down", "combine"]
 KERNEL_SOURCES = {"route": ["route.cu", "route_sm100.cu", "common.cuh"],
                   "pack": ["dispatch.cu", "reroute.cu", "common.cuh"],
-                  "gemm_gate_up": ["gemm_sm100.cu", "common.cuh"],
-                  "gemm_down": ["gemm_sm100.cu", "common.cuh"],
+                  "gemm_gate_up": ["gemm_sm100.cu", "gemm_cols_sm100.cu", "gemm_common.cuh",
+                                   "common.cuh"],
+                  "gemm_down": ["gemm_sm100.cu", "gemm_cols_sm100.cu", "gemm_common.cuh",
+                                "common.cuh"],
                   "combine": ["combine.cu", "common.cuh"]}
 
 
@@ -78,6 +80,11 @@ def parse_args(argv=None):
     ap.add_argument("--stats", action="store_true",
                     help="also gather routing statistics: the router's per-tile sums and one "
                          "moe_routing_stats call per layer")
+    ap.add_argument("--tiles", default="auto", choices=["auto", "rows", "columns"],
+                    help="expert-FFN tile shape (bf16)")
+    ap.add_argument("--fuse", default="none", choices=["none", "gather", "combine", "gather+combine"],
+                    help="steps fused into the expert GEMMs (workloads with the reroute policy "
+                         "or fp32 run unfused)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="launch through the library call by call instead of replaying a CUDA graph")
     a = ap.parse_args(argv)
@@ -318,9 +325,12 @@ def measure_workload(a, wl, dev, world, rank, e2e=False, cpu=False):
     L = wl.layers
     x, layers = I.make_inputs(wl, seed=a.seed + rank, device=dev)
     cap = -1 if wl.phi is None else N.moe_capacity(wl.T, wl.k, wl.E, *wl.phi)
+    fuse = a.fuse if (wl.overflow == "drop" and wl.dtype == "bf16") else "none"
+    tiles = a.tiles if fuse == "none" else "auto"
     cfg = N.make_config(wl.T, wl.d, wl.E, wl.k, wl.d_ff, dtype=wl.dtype, gate_mode=wl.gate_mode,
                         capacity=cap, has_shared=wl.has_shared, add_residual=wl.add_residual,
-                        layout=wl.layout, overflow=wl.overflow, stats=a.stats)
+                        layout=wl.layout, overflow=wl.overflow, stats=a.stats, tiles=tiles,
+                        fuse=fuse)
     ws = N.workspace(cfg, dev)
     summ = torch.zeros((L, 32), dtype=torch.uint8, device=dev)
     ybuf = [torch.empty_like(x), torch.empty_like(x)]
@@ -498,9 +508,12 @@ def measure_workload(a, wl, dev, world, rank, e2e=False, cpu=False):
     breakdown = {k: {"avg_us": round(avg_ms[k] * 1e3, 2), "share": round(tot_ms[k] / sum(tot_ms.values()), 4),
                      "frac": round(roof(k)["frac"], 4), "frac_of_spec": round(roof(k)["frac_of_spec"], 4),
                      "bound": roof(k)["bound"]} for k in KERNELS}
-    launches = L * ((7 if wl.overflow == "reroute" else 5) + int(a.stats))
+    launches = L * ((7 if wl.overflow == "reroute" else 5) + int(a.stats)
+                    - (1 if "combine" in fuse else 0))
 
     out = {"workload": wl.name, "ms_per_step": ms_per_step,
+           "ffn_tiles": N.moe_ffn_tile_shape(cfg) if wl.dtype == "bf16" else "cuda-core",
+           "fuse": fuse,
            "ms_per_step_median": statistics.median(per_step), "value": value, "unit": UNIT,
            "layers": L, "routes_per_step": int(dem.sum()), "kept_rows_per_step": int(sum(Rs)),
            "capacity": cap, "roofline": roofline, "kernels": breakdown, "clocks": clk,
@@ -581,7 +594,8 @@ def run_ours(a):
     for name in a.also:
         r = measure_workload(a, I.WORKLOADS[name], dev, world, rank)
         side[name] = {k: r[k] for k in ("ms_per_step", "value", "unit", "layers",
-                                        "routes_per_step", "capacity", "kernels", "clocks", "l2")}
+                                        "routes_per_step", "capacity", "ffn_tiles", "fuse",
+                                        "kernels", "clocks", "l2")}
         rf = r["roofline"]
         side[name]["roofline"] = {k: rf[k] for k in ("kernel", "bound", "achieved", "peak", "unit",
                                                     "frac", "frac_of_spec", "traffic")}
@@ -594,7 +608,8 @@ def run_ours(a):
               "layers": wl.layers, "gate_mode": wl.gate_mode, "capacity": head["capacity"],
               "shared_expert": wl.has_shared, "residual": wl.add_residual, "layout": wl.layout,
               "overflow": wl.overflow, "routing_stats": a.stats,
-              "parallelism": f"replicas{world}", "cuda_graph": a.graph, "l2": head["l2"]}
+              "parallelism": f"replicas{world}", "cuda_graph": a.graph, "l2": head["l2"],
+              "ffn_tiles": head["ffn_tiles"], "fuse": head["fuse"]}
     out = {
         "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": head["ms_per_step"],

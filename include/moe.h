@@ -82,6 +82,31 @@ typedef enum {
                              * slot (MOE_LAYOUT_PADDED only; see moe_dispatch)              */
 } moe_overflow;
 
+/* Tile shape of the bf16 expert-FFN GEMMs (the fp32 configuration ignores it).  Both give
+ * the same products; they differ in how ragged expert segments are padded.            */
+typedef enum {
+  MOE_TILES_AUTO = 0,    /* row tiles (measured faster than column tiles on every workload
+                          * here), column tiles when a fused step is requested            */
+  MOE_TILES_ROWS = 1,    /* 128 tokens x 256 output columns per tile: tokens on the MMA's M
+                          * side; a segment is padded to a multiple of 128 rows           */
+  MOE_TILES_COLUMNS = 2  /* 128 weight rows x up to 128 tokens per tile: weights on M,
+                          * tokens on N; a segment is padded to a multiple of 16 rows     */
+} moe_tiles;
+
+/* Steps of moe_forward fused into the expert GEMMs (bit flags; bf16, column tiles, drop
+ * overflow policy; the staged calls ignore them).  The results are bit-identical to the
+ * unfused path.  Source: "271,104 Routes...", section 3 (duplicate the token rows, group
+ * them by expert, run the experts, undo the grouping): the copies into and out of the
+ * grouped order are what these flags remove.                                          */
+typedef enum {
+  MOE_FUSE_NONE = 0,
+  MOE_FUSE_GATHER = 1,  /* the gate/up GEMM reads each expert's token rows straight from x
+                         * (by row_token); the pack writes only the route table          */
+  MOE_FUSE_COMBINE = 2  /* the down GEMM's epilogue finishes each output row (gate-weighted
+                         * sum in slot order, shared expert, residual) as soon as its last
+                         * contribution is written; there is no separate combine launch   */
+} moe_fuse;
+
 typedef struct {
   int32_t T;            /* tokens in this call (>= 1)                                   */
   int32_t d;            /* model width                                                   */
@@ -97,6 +122,10 @@ typedef struct {
                          *    tile into the workspace, for moe_routing_stats; 0: off     */
   int32_t layout;       /* moe_layout                                                    */
   int32_t overflow;     /* moe_overflow                                                  */
+  int32_t tiles;        /* moe_tiles (0 = automatic)                                     */
+  int32_t fuse;         /* moe_fuse flags (0 = none); any flag selects column tiles and
+                         * needs MOE_BF16 and MOE_OVERFLOW_DROP (else MOE_ERR_UNSUPPORTED);
+                         * MOE_TILES_ROWS with a flag is MOE_ERR_INVALID                  */
 } moe_config;
 /* Supported shapes (else MOE_ERR_UNSUPPORTED): bf16 needs d % 128 == 0 and
  * d_ff % 128 == 0; fp32 needs d % 4 == 0 and d_ff % 4 == 0.                            */
@@ -116,6 +145,10 @@ int64_t moe_max_rows(const moe_config* cfg);
  * staged calls need only the leading scratch part, which this also covers.
  * Returns 0 for an invalid config.                                                      */
 size_t moe_workspace_bytes(const moe_config* cfg);
+
+/* The FFN tile shape a config runs with: MOE_TILES_ROWS or MOE_TILES_COLUMNS (cfg->tiles,
+ * or the automatic choice when it is MOE_TILES_AUTO); 0 for an invalid config.  Host-only. */
+int32_t moe_ffn_tile_shape(const moe_config* cfg);
 
 /* Zero the status word and scratch header of a workspace (async on `stream`).          */
 moe_status moe_workspace_init(void* ws, moe_stream_t stream);

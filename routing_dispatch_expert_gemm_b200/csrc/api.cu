@@ -27,6 +27,11 @@ moe_status validate_config(const moe_config* c) {
   if ((c->layout != MOE_LAYOUT_RAGGED && c->layout != MOE_LAYOUT_PADDED) ||
       (c->overflow != MOE_OVERFLOW_DROP && c->overflow != MOE_OVERFLOW_REROUTE))
     return MOE_ERR_INVALID;
+  if (c->tiles < MOE_TILES_AUTO || c->tiles > MOE_TILES_COLUMNS) return MOE_ERR_INVALID;
+  if (c->fuse < 0 || c->fuse > (MOE_FUSE_GATHER | MOE_FUSE_COMBINE)) return MOE_ERR_INVALID;
+  if (c->fuse != 0 && c->tiles == MOE_TILES_ROWS) return MOE_ERR_INVALID;
+  if (c->fuse != 0 && (c->dtype != MOE_BF16 || c->overflow != MOE_OVERFLOW_DROP))
+    return MOE_ERR_UNSUPPORTED;
   if (c->layout == MOE_LAYOUT_PADDED && c->capacity < 0) return MOE_ERR_INVALID;  // C sizes it
   if (c->overflow == MOE_OVERFLOW_REROUTE && c->layout != MOE_LAYOUT_PADDED)
     return MOE_ERR_UNSUPPORTED;
@@ -48,7 +53,7 @@ namespace {
 
 moe_status validate(const moe_config* c) { return validate_config(c); }
 
-constexpr int32_t kAbiVersion = 3;
+constexpr int32_t kAbiVersion = 5;
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
@@ -66,7 +71,7 @@ bool reroute(const moe_config& c) { return c.overflow == MOE_OVERFLOW_REROUTE; }
 size_t offsets_len(const moe_config& c) { return c.E + 2 + (padded(c) ? c.E : 0); }
 
 struct Layout {
-  size_t tile_hist, tile_psum, stats_partial, zkeys, rlist;
+  size_t tile_hist, tile_psum, stats_partial, zkeys, rlist, need, counters;
   size_t ids, gates, route_row, row_token, offsets, demand;
   size_t x_packed, h, y_packed;
   size_t scratch_end, total;
@@ -93,6 +98,10 @@ Layout layout_of(const moe_config& c) {
   L.zkeys = reroute(c) ? take(static_cast<size_t>(c.T) * c.E * 4) : 0;
   L.rlist = reroute(c) ? take((2 * static_cast<size_t>(c.E) * c.capacity + 1 +
                                 4 * static_cast<size_t>(c.T) * c.k) * 4) : 0;
+  // Fused combine (MOE_FUSE_COMBINE): contributions per token, counters per 32 columns.
+  L.need = (c.fuse & MOE_FUSE_COMBINE) ? take(static_cast<size_t>(c.T) * 4) : 0;
+  L.counters = (c.fuse & MOE_FUSE_COMBINE) ? take(static_cast<size_t>(c.T) * ((c.d + 31) / 32) * 4)
+                                           : 0;
   L.scratch_end = off;
   L.ids = take(Tk * 4);
   L.gates = take(Tk * 4);
@@ -161,23 +170,38 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
   void* h = at(ws, L.h);
   void* y_packed = at(ws, L.y_packed);
 
+  // The router's last tile also turns the histogram into prefixes and writes the segment
+  // table, so the pack reads finished positions.
+  const DispatchPrep prep = make_dispatch_prep(
+      c, hist, offsets, demand, reinterpret_cast<unsigned int*>(at(ws, kWsPrepCounterOffset)));
   MOE_TRY(record(ev, 0, stream));
   MOE_TRY(cuda_status(
-      launch_router(c, x, w_router, logit_bias, ids, gates, hist, extra, status, stream)));
+      launch_router(c, x, w_router, logit_bias, ids, gates, hist, extra, prep, status, stream)));
   MOE_TRY(record(ev, 1, stream));
-  MOE_TRY(cuda_status(launch_dispatch_scatter(c, x, ids, hist, x_packed, row_token, route_row,
-                                              offsets, demand, status, stream)));
+  const bool fuse_gather = (c.fuse & MOE_FUSE_GATHER) != 0;
+  const bool fuse_combine = (c.fuse & MOE_FUSE_COMBINE) != 0;
+  int32_t* need = fuse_combine ? reinterpret_cast<int32_t*>(at(ws, L.need)) : nullptr;
+  int32_t* counters = fuse_combine ? reinterpret_cast<int32_t*>(at(ws, L.counters)) : nullptr;
+  const void* resid = c.add_residual ? x : nullptr;
+  const PackFusion pf{fuse_gather ? 0 : 1, need, counters, resid, fuse_combine ? y : nullptr,
+                      c.has_shared};
+  MOE_TRY(cuda_status(launch_dispatch_pack(c, x, ids, hist, offsets, x_packed, row_token,
+                                           route_row, status, stream,
+                                           c.fuse != 0 ? &pf : nullptr)));
   if (reroute(c))
     MOE_TRY(cuda_status(launch_reroute(c, x, ids, extra.zkeys, gates, x_packed, row_token,
                                        route_row, offsets,
                                        reinterpret_cast<int32_t*>(at(ws, L.rlist)), status,
                                        stream)));
   MOE_TRY(record(ev, 2, stream));
+  const FusedCombine fc{route_row, gates, row_token, need, counters, resid, y, c.k, c.has_shared};
   FfnArgs f{x, x_packed, offsets, w_gate, w_up, w_down, shared_gate, shared_up, shared_down,
-            h, y_packed, L.rmax, status, padded(c) ? offsets + c.E + 2 : nullptr};
+            h, y_packed, L.rmax, status, padded(c) ? offsets + c.E + 2 : nullptr,
+            fuse_gather ? row_token : nullptr, fuse_combine ? &fc : nullptr};
   MOE_TRY(ffn(c, f, stream, ev ? static_cast<cudaEvent_t>(ev[3]) : nullptr));
   MOE_TRY(record(ev, 4, stream));
-  MOE_TRY(cuda_status(launch_combine(c, y_packed, route_row, gates, offsets, x, y, stream)));
+  if (!fuse_combine)
+    MOE_TRY(cuda_status(launch_combine(c, y_packed, route_row, gates, offsets, x, y, stream)));
   return record(ev, 5, stream);
 }
 
@@ -208,6 +232,11 @@ int32_t moe_capacity(int32_t T, int32_t k, int32_t E, int32_t phi_num, int32_t p
   return c > INT32_MAX ? -1 : static_cast<int32_t>(c);
 }
 
+int32_t moe_ffn_tile_shape(const moe_config* cfg) {
+  if (validate(cfg) != MOE_OK) return 0;
+  return ffn_tile_shape(*cfg);
+}
+
 int64_t moe_max_rows(const moe_config* cfg) {
   if (validate(cfg) != MOE_OK) return 0;
   return max_rows(*cfg);
@@ -232,9 +261,10 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router,
   const Layout L = layout_of(*cfg);
   const RouterExtras extra{cfg->stats ? reinterpret_cast<float*>(at(ws, L.tile_psum)) : nullptr,
                            reroute(*cfg) ? reinterpret_cast<float*>(at(ws, L.zkeys)) : nullptr};
+  const DispatchPrep no_prep{};  // moe_dispatch recounts from the ids it is given
   return cuda_status(launch_router(*cfg, x, w_router, logit_bias, ids, gates,
                                    reinterpret_cast<int32_t*>(at(ws, L.tile_hist)), extra,
-                                   static_cast<int32_t*>(ws), stream));
+                                   no_prep, static_cast<int32_t*>(ws), stream));
 }
 
 moe_status moe_dispatch(const moe_config* cfg, const void* x, const int32_t* ids,
@@ -248,9 +278,11 @@ moe_status moe_dispatch(const moe_config* cfg, const void* x, const int32_t* ids
   const Layout L = layout_of(*cfg);
   int32_t* hist = reinterpret_cast<int32_t*>(at(ws, L.tile_hist));
   int32_t* status = static_cast<int32_t*>(ws);
-  MOE_TRY(cuda_status(launch_dispatch_hist(*cfg, ids, hist, status, stream)));
-  MOE_TRY(cuda_status(launch_dispatch_scatter(*cfg, x, ids, hist, x_packed, row_token, route_row,
-                                              offsets, demand, status, stream)));
+  const DispatchPrep prep = make_dispatch_prep(
+      *cfg, hist, offsets, demand, reinterpret_cast<unsigned int*>(at(ws, kWsPrepCounterOffset)));
+  MOE_TRY(cuda_status(launch_dispatch_hist(*cfg, ids, prep, status, stream)));
+  MOE_TRY(cuda_status(launch_dispatch_pack(*cfg, x, ids, hist, offsets, x_packed, row_token,
+                                           route_row, status, stream)));
   if (!reroute(*cfg)) return MOE_OK;
   return cuda_status(launch_reroute(*cfg, x, ids, reinterpret_cast<const float*>(at(ws, L.zkeys)),
                                     gates, x_packed, row_token, route_row, offsets,

@@ -19,6 +19,9 @@ namespace moe {
 constexpr size_t kWsHeaderBytes = 256;
 // Byte offset, in the header, of the ticket counter of the routing-statistics kernel.
 constexpr size_t kWsStatsCounterOffset = 64;
+// Byte offset, in the header, of the ticket counter of the dispatch prep (the CTA that
+// writes the last tile of the expert histogram turns it into prefixes and offsets).
+constexpr size_t kWsPrepCounterOffset = 128;
 
 // A route (t, j) is valid if its expert id is in range and not repeated earlier in the
 // token's row of ids.

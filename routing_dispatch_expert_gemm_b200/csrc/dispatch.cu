@@ -1,5 +1,5 @@
 // Pack: per-expert demand, arrival-order positions, capacity mask, expert-major offsets,
-// and the scatter of duplicated token rows into expert batches.
+// and the copy of duplicated token rows into expert batches.
 //
 // Sources: "271,104 Routes: What I Missed About Mixture-of-Experts", section 3 Dispatch
 // (route table of token, expert, position, gate; group by expert; bincount + cumsum
@@ -9,31 +9,38 @@
 //
 // Positions are deterministic without ordered atomics: the position of route (t, j) in
 // expert e is the number of earlier tokens that chose e, i.e.
-//   (routes to e in earlier token tiles)  +  popcount(bitmask of earlier tokens of this
-//   tile that chose e).
-// The first term is an exclusive prefix over the per-128-token-tile histogram; every CTA
-// computes the prefix it needs directly from the histogram (ceil(T/128) x E entries), so
-// no separate scan launch and no inter-CTA waiting is needed.  Pack CTAs cover 8-token
-// sub-tiles of a histogram tile, so the copy work spreads over many SMs.  A CTA starts the
-// bulk loads of its token rows first (they do not depend on the routing), works out the
-// positions meanwhile, then all its warps write each row to its kept routes' rows.  With
-// the padded [E, C, d] buffer expert e's rows start at e*C and empty slots are marked -1.
+//   (routes to e in earlier 128-token tiles)  +  (earlier tokens of t's tile that chose e).
+// The first term is the exclusive prefix that the dispatch prep leaves in place of the
+// tile histogram (dispatch_prep.cuh: computed once, by the CTA that writes the histogram's
+// last tile, in the router for moe_forward or in hist_kernel for caller-given ids); the
+// second is counted by the token's warp with ballots over the tile's ids.  Each warp owns
+// one token: it loads the token row while it works out the positions, then writes the row
+// to each kept route's row with 16-byte stores.  With the padded [E, C, d] buffer expert
+// e's rows start at e*C and empty slots are marked -1.
 #include "common.cuh"
+#include "dispatch_prep.cuh"
 #include "internal.h"
 
 namespace moe {
+
+DispatchPrep make_dispatch_prep(const moe_config& c, int32_t* tile_hist, int32_t* offsets,
+                                int32_t* demand, unsigned int* ticket) {
+  return DispatchPrep{tile_hist, offsets, demand, ticket, num_tiles_for(c.T, c.E), c.E, c.T,
+                      c.capacity, c.has_shared, c.layout == MOE_LAYOUT_PADDED ? 1 : 0};
+}
 
 namespace {
 
 constexpr int kThreads = 256;
 
 __global__ void __launch_bounds__(kThreads)
-    hist_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int tok_tile,
-                int32_t* __restrict__ tile_hist, int32_t* status) {
+    hist_kernel(const int32_t* __restrict__ ids, int T, int k, int E, DispatchPrep prep,
+                int32_t* status) {
   __shared__ int s_hist[256];
+  __shared__ int s_scratch[kPrepScratchInts];
   const int tile = blockIdx.x;
-  const int tok0 = tile * tok_tile;
-  const int ntok = min(tok_tile, T - tok0);
+  const int tok0 = tile * kHistTile;
+  const int ntok = min(kHistTile, T - tok0);
   for (int e = threadIdx.x; e < E; e += kThreads) s_hist[e] = 0;
   pdl_trigger();
   pdl_wait();
@@ -49,241 +56,196 @@ __global__ void __launch_bounds__(kThreads)
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += kThreads)
-    tile_hist[static_cast<size_t>(tile) * E + e] = s_hist[e];
+    prep.tile_hist[static_cast<size_t>(tile) * E + e] = s_hist[e];
+  dispatch_prep_arrive(prep, s_scratch);
 }
 
-struct ScatterArgs {
+struct PackArgs {
   const void* x;
   const int32_t* ids;
-  const int32_t* tile_hist;
-  int T, d, k, E, tok_tile, num_tiles, capacity, has_shared, copy_round, padded;
+  const int32_t* tile_prefix;  // [num_tiles, E]: routes to e in earlier tiles
+  const int32_t* offsets;      // segment table ([E+2], or [2E+2] padded)
+  int T, d, k, E, capacity, padded;
   void* x_packed;
   int32_t* row_token;
   int32_t* route_row;
-  int32_t* offsets;
-  int32_t* demand;
   int32_t* status;
+  // fused steps of moe_forward (see PackFusion)
+  int copy;
+  int32_t* need;
+  int32_t* counters;
+  int counter_cols;
+  const void* residual;
+  void* y;
+  int has_shared;
 };
 
-constexpr int kSubTok = 8;  // tokens packed per CTA
-constexpr size_t kStageBudget = 64 * 1024;  // shared memory staging token rows for the copy
+constexpr int kWarpsPerCta = kThreads / 32;
+constexpr int kNV = 8;  // 16-byte vectors per lane per pass over a token row (4 KB per warp)
 
-template <typename T>
-__global__ void __launch_bounds__(kThreads) scatter_kernel(ScatterArgs a) {
-  constexpr int kBatch = 8;    // histogram loads in flight per thread
-  constexpr int kWords = kHistTile / 32;
-  __shared__ int s_pre[256];   // routes to e in earlier tiles
-  __shared__ int s_tot[256];   // routes to e in all tiles (demand)
-  __shared__ int s_off[257];   // segment starts over kept routes
-  __shared__ int s_rows[kSubTok][32];
-  __shared__ uint32_t s_mask[256 * kWords];  // [E][words]: bit = token of the tile chose e
-  __shared__ int s_ids[kHistTile * 32];      // the histogram tile's expert ids [128][k]
-  __shared__ __align__(8) uint64_t s_bar;
-  extern __shared__ __align__(128) uint8_t s_stage[];  // copy_round token rows
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int t_begin = blockIdx.x * kSubTok;
-  const int nsub = min(kSubTok, a.T - t_begin);
-  const int tile = t_begin / kHistTile;
-  const int tile0 = tile * kHistTile;
-  const int ntile = min(kHistTile, a.T - tile0);
-  const int E = a.E, k = a.k;
-
-  for (int e = tid; e < E; e += kThreads) { s_pre[e] = 0; s_tot[e] = 0; }
-  for (int w = tid; w < E * kWords; w += kThreads) s_mask[w] = 0;
+template <typename T, int KMAX>
+__global__ void __launch_bounds__(kThreads) pack_kernel(PackArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_trigger();
   pdl_wait();
-
-  // 0. The token rows do not depend on the routing: start the first round of their bulk
-  //    loads now, so that they arrive while the positions are being worked out.
-  const uint32_t row_bytes = static_cast<uint32_t>(a.d) * sizeof(T);
-  const int round = a.copy_round;  // token rows staged at a time
-  const T* __restrict__ X = static_cast<const T*>(a.x);
-  T* __restrict__ XP = static_cast<T*>(a.x_packed);
-  if (tid == 0) {
-    mbar_init(&s_bar, 1);
-    fence_mbar_init();
-    const int nr = min(round, nsub);
-    mbar_arrive_expect_tx(&s_bar, nr * row_bytes);
-    for (int i = 0; i < nr; ++i)
-      bulk_load(s_stage + i * row_bytes, X + static_cast<size_t>(t_begin + i) * a.d, row_bytes,
-                &s_bar);
-  }
-  // The tile's expert ids, one coalesced pass (its loads overlap the histogram's below).
-  for (int r = tid; r < ntile * k; r += kThreads)
-    s_ids[r] = __ldg(a.ids + static_cast<size_t>(tile0) * k + r);
-  __syncthreads();
-
-  // 1. prefix (tiles < this one) and total per expert, split over all threads with
-  //    kBatch independent loads in flight per thread
-  {
-    const int nparts = kThreads / E;  // >= 1 since E <= 256
-    if (tid < nparts * E) {
-      const int e = tid % E, part = tid / E;
-      int pre = 0, tot = 0;
-      for (int i0 = part; i0 < a.num_tiles; i0 += nparts * kBatch) {
-        int h[kBatch];
-#pragma unroll
-        for (int q = 0; q < kBatch; ++q) {
-          const int i = i0 + q * nparts;
-          h[q] = (i < a.num_tiles) ? __ldg(a.tile_hist + static_cast<size_t>(i) * E + e) : 0;
-        }
-#pragma unroll
-        for (int q = 0; q < kBatch; ++q) {
-          tot += h[q];
-          pre += (i0 + q * nparts < tile) ? h[q] : 0;
-        }
-      }
-      atomicAdd(&s_pre[e], pre);
-      atomicAdd(&s_tot[e], tot);
-    }
-  }
-  // 2. bitmask of the histogram tile's tokens per expert
-  for (int r = tid; r < ntile * k; r += kThreads) {
-    const int tl = r / k, j = r % k;
-    const int32_t* row = s_ids + tl * k;
-    const int e = row[j];
-    if (route_id_valid(row, j, e, E)) atomicOr(&s_mask[e * kWords + (tl >> 5)], 1u << (tl & 31));
-  }
-  __syncthreads();
-
-  // 3. kept counts -> exclusive scan -> offsets (warp 0, 32 experts per step); the padded
-  //    buffer gives expert e the fixed rows e*C ..
-  if (a.padded) {
-    for (int e = tid; e <= E; e += kThreads) s_off[e] = e * a.capacity;
-  } else if (warp == 0) {
-    int carry = 0;
-    for (int base = 0; base < E; base += 32) {
-      const int e = base + lane;
-      int kept = 0;
-      if (e < E) kept = (a.capacity < 0) ? s_tot[e] : min(s_tot[e], a.capacity);
-      int incl = kept;
-#pragma unroll
-      for (int s = 1; s < 32; s <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, incl, s);
-        if (lane >= s) incl += o;
-      }
-      if (e < E) s_off[e] = carry + incl - kept;
-      carry += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) s_off[E] = carry;
-  }
-  __syncthreads();
-  if (blockIdx.x == 0) {
-    for (int e = tid; e <= E; e += kThreads) a.offsets[e] = s_off[e];
-    if (tid == 0) a.offsets[E + 1] = s_off[E] + (a.has_shared ? a.T : 0);
-    for (int e = tid; e < E; e += kThreads) a.demand[e] = s_tot[e];
-    if (a.padded)  // filled slots
-      for (int e = tid; e < E; e += kThreads) a.offsets[E + 2 + e] = min(s_tot[e], a.capacity);
-  }
-  if (a.padded) {  // padding slots of the buffer: row_token = -1 (the CTAs share the sweep)
+  const int E = a.E, k = a.k;
+  if (a.padded) {  // padding slots of the buffer: row_token = -1 (every CTA takes a share)
     const long long slots = static_cast<long long>(E) * a.capacity;
-    for (long long i = static_cast<long long>(blockIdx.x) * kThreads + tid; i < slots;
+    for (long long i = static_cast<long long>(blockIdx.x) * kThreads + threadIdx.x; i < slots;
          i += static_cast<long long>(gridDim.x) * kThreads) {
       const int e = static_cast<int>(i / a.capacity);
       const int p = static_cast<int>(i - static_cast<long long>(e) * a.capacity);
-      if (p >= s_tot[e]) a.row_token[i] = -1;
+      if (p >= __ldg(a.offsets + E + 2 + e)) a.row_token[i] = -1;
     }
   }
+  const int t = blockIdx.x * kWarpsPerCta + warp;
+  if (t >= a.T) return;
 
-  // 4. rows of this CTA's tokens' routes
-  for (int r = tid; r < nsub * k; r += kThreads) {
-    const int ts = r / k, j = r - ts * k;
-    const int t = t_begin + ts, tl = t - tile0;
-    const int32_t* row = s_ids + tl * k;
-    const int e = row[j];
-    int out = -1;
-    if (route_id_valid(row, j, e, E)) {
-      const uint32_t* m = s_mask + e * kWords;
-      int rank = __popc(m[tl >> 5] & ((1u << (tl & 31)) - 1u));
-      for (int w = 0; w < (tl >> 5); ++w) rank += __popc(m[w]);
-      const int pos = s_pre[e] + rank;
-      if (a.capacity < 0 || pos < a.capacity) {
-        out = s_off[e] + pos;
-        a.row_token[out] = t;
-      }
-    }
-    a.route_row[static_cast<size_t>(t) * k + j] = out;
-    s_rows[ts][j] = out;
+  // 1. The first pass of the token row goes out first: it does not depend on the routing.
+  const int nvec = a.d * static_cast<int>(sizeof(T)) / 16;
+  const uint4* __restrict__ xrow = reinterpret_cast<const uint4*>(static_cast<const T*>(a.x) +
+                                                                   static_cast<size_t>(t) * a.d);
+  uint4 v[kNV];
+#pragma unroll
+  for (int i = 0; i < kNV; ++i) {
+    const int idx = i * 32 + lane;
+    v[i] = idx < nvec ? __ldg(xrow + idx) : make_uint4(0, 0, 0, 0);
   }
-  __syncthreads();
 
-  // 5. copy: each token row is loaded once into shared memory by the bulk-copy engine
-  //    (the first round was issued at the start) and written to each of its kept routes'
-  //    rows by all warps with 16-byte stores, one warp per destination row.
-  __shared__ int s_ok;
-  uint32_t phase = 0;
-  const int nvec = static_cast<int>(row_bytes / 16);
-  for (int r0 = 0; r0 < nsub; r0 += round) {
-    const int nr = min(round, nsub - r0);
-    if (r0 > 0) {
-      __syncthreads();  // every warp has finished reading the previous round's rows
-      if (tid == 0) {
-        mbar_arrive_expect_tx(&s_bar, nr * row_bytes);
-        for (int i = 0; i < nr; ++i)
-          bulk_load(s_stage + i * row_bytes, X + static_cast<size_t>(t_begin + r0 + i) * a.d,
-                    row_bytes, &s_bar);
+  // 2. The token's routes: lane j holds slot j.  A route is valid if its id is in range
+  //    and not repeated earlier in the token's row.
+  int e = -1;
+  if (lane < k) e = __ldg(a.ids + static_cast<size_t>(t) * k + lane);
+  bool valid = lane < k && e >= 0 && e < E;
+#pragma unroll
+  for (int q = 0; q < KMAX; ++q) {
+    if (q >= k) break;
+    const int eq = __shfl_sync(0xffffffffu, e, q);
+    if (q < lane && eq == e) valid = false;
+  }
+  if (lane < k && !valid) record_status(a.status, MOE_ERR_BAD_EXPERT_ID);
+  // rank among the earlier tokens of the tile: lane l looks at token c + l; for each slot j
+  // a ballot counts the earlier tokens that hold slot j's expert (once per token, as the
+  // histogram counts it)
+  const int tile = t / kHistTile;
+  int rank = 0;
+  for (int c = tile * kHistTile; c < t; c += 32) {
+    const int tok = c + lane;
+    int row[KMAX];
+#pragma unroll
+    for (int q = 0; q < KMAX; ++q)
+      row[q] = (q < k && tok < t) ? __ldg(a.ids + static_cast<size_t>(tok) * k + q) : -1;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      if (j >= k) break;
+      const int ej = __shfl_sync(0xffffffffu, e, j);
+      const bool vj = __shfl_sync(0xffffffffu, valid ? 1 : 0, j) != 0;
+      bool m = false;
+#pragma unroll
+      for (int q = 0; q < KMAX; ++q) m |= (row[q] == ej);
+      const int cnt = __popc(__ballot_sync(0xffffffffu, vj && m));
+      if (lane == j) rank += cnt;
+    }
+  }
+  int out = -1;
+  if (valid) {
+    const int pos = __ldg(a.tile_prefix + static_cast<size_t>(tile) * E + e) + rank;
+    if (a.capacity < 0 || pos < a.capacity) {
+      out = a.padded ? e * a.capacity + pos : __ldg(a.offsets + e) + pos;
+      a.row_token[out] = t;
+    }
+  }
+  if (lane < k) a.route_row[static_cast<size_t>(t) * k + lane] = out;
+
+  // Fused combine: the token's number of contributions and its zeroed counters; a token
+  // with none (every route dropped, no shared expert) gets its output row here:
+  // x[t] with the residual, else zeros (what the combine's fp32 sum would round to).
+  bool write_y = false;
+  if (a.need != nullptr) {
+    const int cnt = __popc(__ballot_sync(0xffffffffu, lane < k && out >= 0)) + a.has_shared;
+    if (lane == 0) a.need[t] = cnt;
+    for (int i = lane; i < a.counter_cols; i += 32)
+      a.counters[static_cast<size_t>(t) * a.counter_cols + i] = 0;
+    write_y = (cnt == 0);
+  }
+  if (!a.copy && !write_y) return;
+
+  // 3. Copy: each pass of the row is written to every kept route's row.
+  T* __restrict__ XP = static_cast<T*>(a.x_packed);
+  uint4* __restrict__ yrow = write_y ? reinterpret_cast<uint4*>(static_cast<T*>(a.y) +
+                                                                 static_cast<size_t>(t) * a.d)
+                                     : nullptr;
+  for (int base = 0; base < nvec; base += 32 * kNV) {
+    if (base > 0) {
+#pragma unroll
+      for (int i = 0; i < kNV; ++i) {
+        const int idx = base + i * 32 + lane;
+        v[i] = idx < nvec ? __ldg(xrow + idx) : make_uint4(0, 0, 0, 0);
       }
     }
-    if (tid == 0) {
-      int ok = mbar_wait_bounded(&s_bar, phase, nullptr, kWaitLimitNs, a.status);
-      if (!ok) mbar_wait_bounded(&s_bar, phase, nullptr, kWaitLimitNs, a.status);  // drain
-      s_ok = ok;
+    if (write_y) {
+#pragma unroll
+      for (int i = 0; i < kNV; ++i) {
+        const int idx = base + i * 32 + lane;
+        if (idx < nvec) yrow[idx] = a.residual != nullptr ? v[i] : make_uint4(0, 0, 0, 0);
+      }
     }
-    __syncthreads();  // the rows have landed (thread 0 saw the transaction count complete)
-    if (!s_ok) return;
-    phase ^= 1u;
-    for (int ij = warp; ij < nr * k; ij += kThreads / 32) {
-      const int i = ij / k, j = ij - i * k;
-      const int r = s_rows[r0 + i][j];
+    if (!a.copy) continue;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      if (j >= k) break;
+      const int r = __shfl_sync(0xffffffffu, out, j);
       if (r < 0) continue;
-      const uint4* src = reinterpret_cast<const uint4*>(s_stage + i * row_bytes);
       uint4* dst = reinterpret_cast<uint4*>(XP + static_cast<size_t>(r) * a.d);
-      for (int v = lane; v < nvec; v += 32) dst[v] = src[v];
+#pragma unroll
+      for (int i = 0; i < kNV; ++i) {
+        const int idx = base + i * 32 + lane;
+        if (idx < nvec) dst[idx] = v[i];
+      }
     }
   }
+}
+
+template <typename T>
+cudaError_t launch_pack_typed(const PackArgs& a, cudaStream_t s) {
+  const int grid = (a.T + kWarpsPerCta - 1) / kWarpsPerCta;
+  const dim3 g(grid), b(kThreads);
+  if (a.k <= 1) return launch_pdl(pack_kernel<T, 1>, g, b, 0, s, a);
+  if (a.k <= 2) return launch_pdl(pack_kernel<T, 2>, g, b, 0, s, a);
+  if (a.k <= 4) return launch_pdl(pack_kernel<T, 4>, g, b, 0, s, a);
+  if (a.k <= 8) return launch_pdl(pack_kernel<T, 8>, g, b, 0, s, a);
+  if (a.k <= 16) return launch_pdl(pack_kernel<T, 16>, g, b, 0, s, a);
+  return launch_pdl(pack_kernel<T, 32>, g, b, 0, s, a);
 }
 
 }  // namespace
 
-cudaError_t launch_dispatch_hist(const moe_config& c, const int32_t* ids, int32_t* tile_hist,
-                                 int32_t* status, cudaStream_t s) {
-  const int tt = tok_tile_for(c.T, c.E);
-  const int grid = (c.T + tt - 1) / tt;
+cudaError_t launch_dispatch_hist(const moe_config& c, const int32_t* ids,
+                                 const DispatchPrep& prep, int32_t* status, cudaStream_t s) {
+  const int grid = num_tiles_for(c.T, c.E);
   static DeviceOnce once;
   cudaError_t e = once.run([] { return prefer_max_shared(hist_kernel); });
   if (e != cudaSuccess) return e;
-  return launch_pdl(hist_kernel, dim3(grid), dim3(kThreads), 0, s, ids, c.T, c.k, c.E, tt,
-                    tile_hist, status);
+  return launch_pdl(hist_kernel, dim3(grid), dim3(kThreads), 0, s, ids, c.T, c.k, c.E, prep,
+                    status);
 }
 
-cudaError_t launch_dispatch_scatter(const moe_config& c, const void* x, const int32_t* ids,
-                                    const int32_t* tile_hist, void* x_packed,
-                                    int32_t* row_token, int32_t* route_row, int32_t* offsets,
-                                    int32_t* demand, int32_t* status, cudaStream_t s) {
-  const int grid = (c.T + kSubTok - 1) / kSubTok;
-  const size_t row_bytes = static_cast<size_t>(c.d) * (c.dtype == MOE_BF16 ? 2 : 4);
-  int round = static_cast<int>(kStageBudget / row_bytes);
-  round = round < 1 ? 1 : (round > kSubTok ? kSubTok : round);
-  ScatterArgs a{x, ids, tile_hist, c.T, c.d, c.k, c.E, kHistTile, num_tiles_for(c.T, c.E),
-                c.capacity, c.has_shared, round, c.layout == MOE_LAYOUT_PADDED ? 1 : 0, x_packed,
-                row_token, route_row, offsets, demand, status};
-  const size_t smem = static_cast<size_t>(round) * row_bytes;
-  static DeviceOnce once;
-  cudaError_t e = once.run([] {
-    prefer_max_shared(scatter_kernel<__nv_bfloat16>);
-    prefer_max_shared(scatter_kernel<float>);
-    cudaError_t r = cudaFuncSetAttribute(scatter_kernel<__nv_bfloat16>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kStageBudget));
-    if (r != cudaSuccess) return r;
-    return cudaFuncSetAttribute(scatter_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(kStageBudget));
-  });
-  if (e != cudaSuccess) return e;
-  if (c.dtype == MOE_BF16)
-    return launch_pdl(scatter_kernel<__nv_bfloat16>, dim3(grid), dim3(kThreads), smem, s, a);
-  return launch_pdl(scatter_kernel<float>, dim3(grid), dim3(kThreads), smem, s, a);
+cudaError_t launch_dispatch_pack(const moe_config& c, const void* x, const int32_t* ids,
+                                 const int32_t* tile_prefix, const int32_t* offsets,
+                                 void* x_packed, int32_t* row_token, int32_t* route_row,
+                                 int32_t* status, cudaStream_t s, const PackFusion* fused) {
+  PackArgs a{x, ids, tile_prefix, offsets, c.T, c.d, c.k, c.E, c.capacity,
+             c.layout == MOE_LAYOUT_PADDED ? 1 : 0, x_packed, row_token, route_row, status,
+             1, nullptr, nullptr, (c.d + 31) / 32, nullptr, nullptr, c.has_shared};
+  if (fused != nullptr) {
+    a.copy = fused->copy;
+    a.need = fused->need;
+    a.counters = fused->counters;
+    a.residual = fused->residual;
+    a.y = fused->y;
+  }
+  if (c.dtype == MOE_BF16) return launch_pack_typed<__nv_bfloat16>(a, s);
+  return launch_pack_typed<float>(a, s);
 }
 
 }  // namespace moe

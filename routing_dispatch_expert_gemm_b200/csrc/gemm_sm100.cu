@@ -24,10 +24,7 @@
 // Every wait is bounded (mbar_wait_bounded): if one runs out, the CTA records
 // MOE_ERR_TIMEOUT, drains its own copies and MMAs, frees its tensor memory and returns.
 // No TMA multicast is used.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include "common.cuh"
+#include "gemm_common.cuh"
 #include "internal.h"
 
 namespace moe {
@@ -57,8 +54,13 @@ bool encode_2d_box(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows
 
 namespace {
 
+using gemm::BK;
+using gemm::kMaxSeg;
+using gemm::find_seg;
+using gemm::pack_bf16;
+using gemm::silu_f;
+
 constexpr int BM = 128;
-constexpr int BK = 64;  // 64 bf16 = one 128-byte swizzle row
 constexpr int kEpiWarps = 8;                    // two per TMEM lane quarter
 constexpr int kProducerWarp = kEpiWarps;        // warp 8
 constexpr int kMmaWarp = kEpiWarps + 1;         // warp 9
@@ -67,7 +69,6 @@ constexpr int kStageRowBytes = 80;              // 64 B of a row chunk + 16 B pa
 constexpr int kEpiStageBytes = 32 * kStageRowBytes;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int kBoxRows = 128;
-constexpr int kMaxSeg = 260;
 
 struct Maps {
   CUtensorMap a_routed;   // packed rows (gate/up) or H (down): [rows, K]
@@ -98,25 +99,6 @@ struct Cfg {
   static constexpr int SMEM =
       1024 + STAGES * STAGE_BYTES + kEpiWarps * kEpiStageBytes + 256 + 3 * kMaxSeg * 4;
 };
-
-__device__ __forceinline__ int find_seg(const int* pre, int nseg, int tile) {
-  int lo = 0, hi = nseg - 1;  // largest s with pre[s] <= tile
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (pre[mid] <= tile) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
-
-// SiLU(g) = g / (1 + e^-g) with the fast approximate exponential and division (about 2 ulp
-// in fp32; the result is rounded to bf16).  For g -> -inf the denominator overflows and the
-// quotient is 0, the limit of SiLU.
-__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.f + __expf(-g)); }
-
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
 
 template <int MODE, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -162,28 +144,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   pdl_trigger();
   pdl_wait();  // offsets, A rows and the output buffer belong to earlier kernels
-  if (warp == 0) {  // segment table: row starts and exclusive prefix of tile counts
-    for (int i = lane; i <= p.nseg; i += 32) s_row0[i] = __ldg(p.offsets + i);
-    __syncwarp();
-    for (int i = lane; i < p.nseg; i += 32)
-      s_rows[i] = (p.counts != nullptr && i < p.E) ? __ldg(p.counts + i) : s_row0[i + 1] - s_row0[i];
-    __syncwarp();
-    int carry = 0;
-    for (int b = 0; b < p.nseg; b += 32) {
-      const int s = b + lane;
-      int t = 0;
-      if (s < p.nseg) t = ((s_rows[s] + BM - 1) / BM) * n_blocks;
-      int incl = t;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      if (s < p.nseg) s_pre[s] = carry + incl - t;
-      carry += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) s_pre[p.nseg] = carry;
-  }
+  if (warp == 0)  // segment table: row starts and exclusive prefix of tile counts
+    gemm::build_segment_table(p.offsets, p.counts, p.nseg, p.E, BM, n_blocks, s_pre, s_row0,
+                              s_rows);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -366,16 +329,6 @@ bool encode_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows) {
   return encode_2d_box(m, ptr, cols, rows, kBoxRows);
 }
 
-// SMs of the current device (a cheap host query, made per launch so that every device
-// gets its own count).
-int sm_count() {
-  int dev = 0, v = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
-    return 148;
-  return v;
-}
-
 template <int MODE, int BN>
 cudaError_t launch_gemm(const Maps& maps, const Params& p, long long tiles_bound, cudaStream_t s) {
   using C = Cfg<MODE, BN>;
@@ -394,8 +347,31 @@ cudaError_t launch_gemm(const Maps& maps, const Params& p, long long tiles_bound
 
 }  // namespace
 
+// SMs of the current device (a cheap host query, made per launch so that every device
+// gets its own count).
+int sm_count() {
+  int dev = 0, v = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+    return 148;
+  return v;
+}
+
+// Automatic tile shape: row tiles.  Column tiles cut the padding of small expert segments
+// (a 130-row segment costs 256 rows of row-tile MMA work but 144 token columns), but their
+// N <= 128 MMAs read about a third more shared memory per FLOP than the row tiles' N = 256
+// ones, and on B200 that costs more than the padding saves on every workload measured here
+// (the 64+1 layer at T = 4096, the Granite- and Mixtral-shaped layers, decode).  They stay
+// selectable, and they carry the fused gather and combine.
+int32_t ffn_tile_shape(const moe_config& c) {
+  if (c.fuse != 0) return MOE_TILES_COLUMNS;  // the fused steps live in the column kernel
+  if (c.tiles == MOE_TILES_COLUMNS) return MOE_TILES_COLUMNS;
+  return MOE_TILES_ROWS;
+}
+
 cudaError_t launch_ffn_sm100(const moe_config& c, const FfnArgs& f, cudaStream_t s,
                              cudaEvent_t mid) {
+  if (ffn_tile_shape(c) == MOE_TILES_COLUMNS) return launch_ffn_cols_sm100(c, f, s, mid);
   const int nseg = c.E + (c.has_shared ? 1 : 0);
   const long long rows_h = f.rmax + (c.has_shared ? c.T : 0);
   const long long mt_bound = (rows_h + BM - 1) / BM + nseg;

@@ -26,15 +26,32 @@ struct RouterExtras {
                      // top-k compared (the reroute policy ranks with them)
 };
 
+// What the CTA that writes the last tile of the expert histogram computes for the pack
+// (dispatch_prep.cuh): per-tile exclusive prefixes in place of the counts, demand, the
+// segment table (offsets, [E + 2] or [2E + 2] padded) and the filled-slot counts.
+// `ticket` must be zero before the launch; it is left zero.  A null ticket: not computed.
+struct DispatchPrep {
+  int32_t* tile_hist;
+  int32_t* offsets;
+  int32_t* demand;
+  unsigned int* ticket;
+  int num_tiles, E, T, capacity, has_shared, padded;
+};
+DispatchPrep make_dispatch_prep(const moe_config& c, int32_t* tile_hist, int32_t* offsets,
+                                int32_t* demand, unsigned int* ticket);
+
+// Router: ids, gates and the per-tile expert histogram; with a non-null prep.ticket also
+// the dispatch prep above (moe_forward passes one; moe_route does not).
 cudaError_t launch_router(const moe_config& c, const void* x, const void* w_router,
                           const float* bias, int32_t* ids, float* gates, int32_t* tile_hist,
-                          const RouterExtras& extra, int32_t* status, cudaStream_t s);
+                          const RouterExtras& extra, const DispatchPrep& prep, int32_t* status,
+                          cudaStream_t s);
 
 // bf16 router on tensor cores (route_sm100.cu); the fp32 router runs on CUDA cores.
 cudaError_t launch_router_sm100(const moe_config& c, const void* x, const void* w_router,
                                 const float* bias, int32_t* ids, float* gates,
                                 int32_t* tile_hist, const RouterExtras& extra,
-                                int32_t* status, cudaStream_t s);
+                                const DispatchPrep& prep, int32_t* status, cudaStream_t s);
 
 // Routing statistics from the per-tile probability sums and the dispatch counts.
 // partial: [kStatsMaxBlocks, E] fp64 scratch; counter: zero before the call, left zero.
@@ -56,17 +73,47 @@ cudaError_t launch_reroute(const moe_config& c, const void* x, const int32_t* id
                            int32_t* route_row, int32_t* offsets, int32_t* scratch,
                            int32_t* status, cudaStream_t s);
 
-cudaError_t launch_dispatch_hist(const moe_config& c, const int32_t* ids, int32_t* tile_hist,
-                                 int32_t* status, cudaStream_t s);
+// Expert histogram of caller-given ids per 128-token tile (invalid ids are flagged and not
+// counted), followed by the dispatch prep in the last CTA.
+cudaError_t launch_dispatch_hist(const moe_config& c, const int32_t* ids,
+                                 const DispatchPrep& prep, int32_t* status, cudaStream_t s);
 
-cudaError_t launch_dispatch_scatter(const moe_config& c, const void* x, const int32_t* ids,
-                                    const int32_t* tile_hist, void* x_packed,
-                                    int32_t* row_token, int32_t* route_row, int32_t* offsets,
-                                    int32_t* demand, int32_t* status, cudaStream_t s);
+// Pack: route_row, row_token and the packed rows, from the ids and the prep's prefixes and
+// segment table (one warp per token).  With `fused` (moe_forward's fused steps): no row
+// copy when the GEMM gathers (fused->copy == 0); with the fused combine, need[t] and the
+// zeroed counters, and y[t] for tokens with no contribution at all.
+struct PackFusion {
+  int copy;               // 1: write x_packed
+  int32_t* need;          // [T] or null
+  int32_t* counters;      // [T, d / 32] or null
+  const void* residual;   // x or null
+  void* y;                // y (tokens with need 0) or null
+  int has_shared;
+};
+cudaError_t launch_dispatch_pack(const moe_config& c, const void* x, const int32_t* ids,
+                                 const int32_t* tile_prefix, const int32_t* offsets,
+                                 void* x_packed, int32_t* row_token, int32_t* route_row,
+                                 int32_t* status, cudaStream_t s,
+                                 const PackFusion* fused = nullptr);
 
 cudaError_t launch_combine(const moe_config& c, const void* y_packed, const int32_t* route_row,
                            const float* gates, const int32_t* offsets, const void* residual,
                            void* y, cudaStream_t s);
+
+// The combine done in the down GEMM's epilogue (MOE_FUSE_COMBINE): every tile that writes
+// 32 columns of a packed row counts itself on the token's counter for that column chunk;
+// the one that brings it to need[t] (kept routes + shared expert) sums the token's rows
+// of y_packed for those columns in slot order and writes them to y.
+struct FusedCombine {
+  const int32_t* route_row;  // [T, k]
+  const float* gates;        // [T, k]
+  const int32_t* row_token;  // [Rmax] token of each packed row
+  const int32_t* need;       // [T] contributions per token (pack writes it)
+  int32_t* counters;         // [T, d / 32], zeroed by the pack
+  const void* residual;      // x [T, d] or null
+  void* y;                   // [T, d]
+  int k, has_shared;
+};
 
 struct FfnArgs {
   const void* x;          // [T, d] (shared expert's A operand)
@@ -84,15 +131,25 @@ struct FfnArgs {
   int32_t* status;
   const int32_t* counts;  // [E] rows of each routed segment (padded layout), or null:
                           // rows = offsets[s + 1] - offsets[s]
+  // Fused steps (column tiles only; null: not fused).
+  const int32_t* gather_rows;  // row_token [Rmax]: the gate/up GEMM reads x[row_token[r]]
+                               // instead of x_packed[r]
+  const FusedCombine* combine; // the down GEMM's epilogue finishes the output rows
 };
 
 // fp32 path: CUDA-core grouped GEMMs.  `mid` (may be null) is recorded between the
 // gate/up and the down GEMM.
 cudaError_t launch_ffn_simt(const moe_config& c, const FfnArgs& a, cudaStream_t s,
                             cudaEvent_t mid = nullptr);
-// bf16 path: persistent tcgen05/TMEM grouped GEMMs fed by TMA.
+// bf16 path: persistent tcgen05/TMEM grouped GEMMs fed by TMA.  Chooses the tile shape:
+// row tiles (tokens on the MMA's M side, gemm_sm100.cu) for large expert segments, column
+// tiles (weights on M, tokens on N, gemm_cols_sm100.cu) for small ones.
 cudaError_t launch_ffn_sm100(const moe_config& c, const FfnArgs& a, cudaStream_t s,
                              cudaEvent_t mid = nullptr);
+// MOE_TILES_ROWS or MOE_TILES_COLUMNS: cfg.tiles, or the automatic choice.
+int32_t ffn_tile_shape(const moe_config& c);
+cudaError_t launch_ffn_cols_sm100(const moe_config& c, const FfnArgs& a, cudaStream_t s,
+                                  cudaEvent_t mid = nullptr);
 
 cudaError_t launch_debug_wait(int32_t* status, int64_t limit_ns, cudaStream_t s);
 

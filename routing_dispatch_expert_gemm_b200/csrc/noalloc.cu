@@ -15,9 +15,11 @@ namespace moe {
 namespace {
 
 // Largest histogram this entry point handles: num_tiles(T, E) * E int32 entries.  The
-// array lives in every device that loads the library, until the process exits.
+// array holds the histogram and, after it, the ticket counter of the dispatch prep; it
+// lives in every device that loads the library, until the process exits.
 constexpr int kNoAllocHistEntries = 16384;  // 64 KiB
-static __device__ __align__(256) int32_t g_noalloc_hist[kNoAllocHistEntries];
+constexpr int kNoAllocTicket = kNoAllocHistEntries;  // one more 256-byte-aligned slot
+static __device__ __align__(256) int32_t g_noalloc_hist[kNoAllocHistEntries + 64];
 
 // Device address of g_noalloc_hist in the current device's context.  In host code the
 // symbol names a host-side stand-in, not device memory, so the address is looked up with
@@ -55,11 +57,15 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_config* cfg, const void* x,
     return MOE_ERR_UNSUPPORTED;
   int32_t* hist = nullptr;
   if (hist_address(&hist) != cudaSuccess) return MOE_ERR_CUDA;
-  // Nothing in the array has to start at zero: the histogram kernel writes every entry
-  // that the scatter kernel reads.
-  if (launch_dispatch_hist(*cfg, ids, hist, status, stream) != cudaSuccess) return MOE_ERR_CUDA;
-  if (launch_dispatch_scatter(*cfg, x, ids, hist, x_packed, row_token, route_row, offsets,
-                              demand, status, stream) != cudaSuccess)
+  // The histogram kernel writes every histogram entry the pack reads; only the ticket has
+  // to start at zero.  It is cleared here (the prep also leaves it zero), so a call never
+  // depends on what an earlier one left behind.
+  unsigned int* ticket = reinterpret_cast<unsigned int*>(hist + kNoAllocTicket);
+  if (cudaMemsetAsync(ticket, 0, sizeof(unsigned int), stream) != cudaSuccess) return MOE_ERR_CUDA;
+  const DispatchPrep prep = make_dispatch_prep(*cfg, hist, offsets, demand, ticket);
+  if (launch_dispatch_hist(*cfg, ids, prep, status, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_dispatch_pack(*cfg, x, ids, hist, offsets, x_packed, row_token, route_row, status,
+                           stream) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
 }

@@ -16,6 +16,7 @@
 #include <cfloat>
 
 #include "common.cuh"
+#include "dispatch_prep.cuh"
 #include "internal.h"
 
 namespace moe {
@@ -39,6 +40,7 @@ struct RouterArgs {
   int32_t* tile_hist;
   float* tile_psum;  // null: no routing statistics
   float* zkeys;      // null: ranking keys not stored
+  DispatchPrep prep; // null ticket: no dispatch prep
 };
 
 // NaN logits rank as -inf so that k valid experts are always selected.
@@ -244,6 +246,8 @@ __global__ void __launch_bounds__(kThreads, 1) router_kernel(RouterArgs a) {
       for (int w = 0; w < 8; ++w) v += s_psum[w][e];
       a.tile_psum[static_cast<size_t>(tile) * a.E + e] = v;
     }
+  // the probability sums' shared memory is free now: scratch for the dispatch prep
+  if (a.prep.ticket != nullptr) dispatch_prep_arrive(a.prep, reinterpret_cast<int*>(&s_psum[0][0]));
 }
 
 template <typename Tin, int EP>
@@ -282,11 +286,13 @@ cudaError_t launch_typed(RouterArgs a, cudaStream_t s) {
 
 cudaError_t launch_router(const moe_config& c, const void* x, const void* w_router,
                           const float* bias, int32_t* ids, float* gates, int32_t* tile_hist,
-                          const RouterExtras& extra, int32_t* status, cudaStream_t s) {
+                          const RouterExtras& extra, const DispatchPrep& prep, int32_t* status,
+                          cudaStream_t s) {
   if (c.dtype == MOE_BF16)
-    return launch_router_sm100(c, x, w_router, bias, ids, gates, tile_hist, extra, status, s);
+    return launch_router_sm100(c, x, w_router, bias, ids, gates, tile_hist, extra, prep, status,
+                               s);
   RouterArgs a{x, w_router, bias, c.T, c.d, c.E, c.k, c.gate_mode, kHistTile, 0,
-               ids, gates, tile_hist, extra.tile_psum, extra.zkeys};
+               ids, gates, tile_hist, extra.tile_psum, extra.zkeys, prep};
   return launch_typed<float>(a, s);
 }
 

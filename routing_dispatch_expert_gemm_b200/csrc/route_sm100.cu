@@ -25,6 +25,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "dispatch_prep.cuh"
 #include "internal.h"
 
 namespace moe {
@@ -56,6 +57,7 @@ struct RouteParams {
   float* zkeys;      // null: ranking keys not stored
   int32_t* status;
   int64_t limit_ns;
+  DispatchPrep prep; // null ticket: no dispatch prep
 };
 
 __device__ __forceinline__ float rank_key(float z) { return isnan(z) ? -INFINITY : z; }
@@ -363,6 +365,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 5) tmem_dealloc(tmem_base, p.tmem_cols);
+  // the TMA ring is idle now: scratch for the dispatch prep
+  if (p.prep.ticket != nullptr) dispatch_prep_arrive(p.prep, reinterpret_cast<int*>(base));
 }
 
 // ---------------------------------------------------------------------------------
@@ -642,6 +646,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 5) tmem_dealloc(tmem_base, p.tmem_cols);
+  // One arrival per tile (CTA 0 wrote its histogram row).  No CTA of the cluster reads the
+  // partial-logit array any more: it is scratch for the dispatch prep.
+  if (rank == 0 && p.prep.ticket != nullptr)
+    dispatch_prep_arrive(p.prep, reinterpret_cast<int*>(s_part));
 }
 
 template <int EN_T>
@@ -688,7 +696,7 @@ cudaError_t launch_en(const RouteMaps& maps, const RouteParams& p, int grid, int
 cudaError_t launch_router_sm100(const moe_config& c, const void* x, const void* w_router,
                                 const float* bias, int32_t* ids, float* gates,
                                 int32_t* tile_hist, const RouterExtras& extra,
-                                int32_t* status, cudaStream_t s) {
+                                const DispatchPrep& prep, int32_t* status, cudaStream_t s) {
   float* tile_psum = extra.tile_psum;
   // Logit columns (MMA N): 16, 32 or 64 when E fits, so the epilogue can keep a token's
   // logits in registers; otherwise E rounded up to a multiple of 16.
@@ -705,7 +713,7 @@ cudaError_t launch_router_sm100(const moe_config& c, const void* x, const void* 
       !encode_2d_box(&maps.w, w_router, c.d, c.E, EN))
     return cudaErrorInvalidValue;
   RouteParams p{bias, c.T, c.d, c.E, c.k, EN, c.gate_mode, stages, cols,
-                ids, gates, tile_hist, tile_psum, extra.zkeys, status, kWaitLimitNs};
+                ids, gates, tile_hist, tile_psum, extra.zkeys, status, kWaitLimitNs, prep};
   const int ntiles = (c.T + kTokens - 1) / kTokens;
   if (EN <= 64 && k_blocks >= kCluster) {
     // one 128-token tile per cluster of 8 CTAs, each with 1/8 of d

@@ -13,7 +13,7 @@ import os
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
 
 MOE_OK = 0
-ABI_VERSION = 3  # moe_abi_version() of the library this binding mirrors
+ABI_VERSION = 5  # moe_abi_version() of the library this binding mirrors
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID", 2: "MOE_ERR_UNSUPPORTED",
                 3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_BAD_EXPERT_ID",
                 6: "MOE_ERR_TIMEOUT"}
@@ -21,9 +21,12 @@ DTYPES = {"f32": 0, "bf16": 1}
 GATE_MODES = {"softmax_topk": 0, "softmax_topk_renorm": 1, "topk_softmax": 2}
 LAYOUTS = {"ragged": 0, "padded": 1}
 OVERFLOWS = {"drop": 0, "reroute": 1}
+TILES = {"auto": 0, "rows": 1, "columns": 2}
+FUSE = {"none": 0, "gather": 1, "combine": 2, "gather+combine": 3}
 
 # Every symbol include/moe.h declares (checked by the CPU test suite).
 EXPORTS = ("moe_capacity", "moe_max_rows", "moe_workspace_bytes", "moe_workspace_init",
+           "moe_ffn_tile_shape",
            "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_forward_profiled", "moe_get_device_status", "moe_debug_bounded_wait",
            "moe_dispatch_noalloc", "moe_routing_stats", "moe_status_string",
@@ -39,7 +42,8 @@ class MoeError(RuntimeError):
 class MoeConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("T", "d", "E", "k", "d_ff", "dtype", "gate_mode", "capacity",
-                 "has_shared", "add_residual", "stats", "layout", "overflow")]
+                 "has_shared", "add_residual", "stats", "layout", "overflow", "tiles",
+                 "fuse")]
 
     def __repr__(self):
         return "MoeConfig(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
@@ -47,11 +51,11 @@ class MoeConfig(ctypes.Structure):
 
 def make_config(T, d, E, k, d_ff, dtype="bf16", gate_mode="topk_softmax", capacity=-1,
                 has_shared=False, add_residual=False, stats=False, layout="ragged",
-                overflow="drop") -> MoeConfig:
+                overflow="drop", tiles="auto", fuse="none") -> MoeConfig:
     return MoeConfig(int(T), int(d), int(E), int(k), int(d_ff), DTYPES[dtype],
                      GATE_MODES[gate_mode], int(capacity), int(bool(has_shared)),
                      int(bool(add_residual)), int(bool(stats)), LAYOUTS[layout],
-                     OVERFLOWS[overflow])
+                     OVERFLOWS[overflow], TILES[tiles], FUSE[fuse])
 
 
 def offsets_len(cfg: MoeConfig) -> int:
@@ -94,6 +98,7 @@ def lib() -> ctypes.CDLL:
             "moe_max_rows": (ctypes.c_int64, [_CFG]),
             "moe_workspace_bytes": (ctypes.c_size_t, [_CFG]),
             "moe_workspace_init": (_I32, [_P, _P]),
+            "moe_ffn_tile_shape": (_I32, [_CFG]),
             "moe_route": (_I32, [_CFG, _P, _P, _P, _P, _P, _P, _P]),
             "moe_dispatch": (_I32, [_CFG] + [_P] * 10),
             "moe_expert_ffn": (_I32, [_CFG] + [_P] * 12 + [_P]),
@@ -155,6 +160,14 @@ def moe_capacity(T, k, E, phi_num, phi_den) -> int:
 
 def moe_max_rows(cfg: MoeConfig) -> int:
     return lib().moe_max_rows(ctypes.byref(cfg))
+
+
+def moe_ffn_tile_shape(cfg: MoeConfig) -> str:
+    """'rows' or 'columns': the FFN tile shape the config runs with."""
+    v = lib().moe_ffn_tile_shape(ctypes.byref(cfg))
+    if v == 0:
+        raise MoeError(1, "moe_ffn_tile_shape")
+    return {1: "rows", 2: "columns"}[v]
 
 
 def moe_workspace_bytes(cfg: MoeConfig) -> int:

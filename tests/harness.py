@@ -19,13 +19,15 @@ def oracle_capacity(wl: I.Workload):
     return None if wl.phi is None else O.capacity(wl.T, wl.k, wl.E, *wl.phi)
 
 
-def config_for(wl: I.Workload, capacity=None, stats=False) -> N.MoeConfig:
+def config_for(wl: I.Workload, capacity=None, stats=False, tiles="auto",
+               fuse="none") -> N.MoeConfig:
     """The GPU-side config; capacity from the library's own moe_capacity."""
     if capacity is None:
         capacity = -1 if wl.phi is None else N.moe_capacity(wl.T, wl.k, wl.E, *wl.phi)
     return N.make_config(wl.T, wl.d, wl.E, wl.k, wl.d_ff, dtype=wl.dtype, gate_mode=wl.gate_mode,
                          capacity=capacity, has_shared=wl.has_shared, add_residual=wl.add_residual,
-                         stats=stats, layout=wl.layout, overflow=wl.overflow)
+                         stats=stats, layout=wl.layout, overflow=wl.overflow, tiles=tiles,
+                         fuse=fuse)
 
 
 def oracle_params(p: dict) -> dict:

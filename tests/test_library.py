@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(native):
     lib = ctypes.CDLL(native.LIB_PATH)
     for name in declared:
         assert hasattr(lib, name), name
-    assert native.moe_abi_version() == native.ABI_VERSION == 3
+    assert native.moe_abi_version() == native.ABI_VERSION == 5
 
 
 def test_library_is_sm100a_build(native):
@@ -193,3 +193,23 @@ def test_config_sweep_validation_and_sizes(native):
             assert rows == max(min(T * k, E * cap) if cap >= 0 else T * k, 1)
         base = native.make_config(T, d, E, k, F, dtype=dtype, capacity=cap, layout=layout)
         assert native.moe_workspace_bytes(base) <= ws
+
+
+def test_ffn_tile_shape_choice(native):
+    """Automatic tile shape: row tiles; column tiles when asked for or when a fused step is
+    requested; bad values and row tiles with fusion rejected."""
+    mk = native.make_config
+    assert native.moe_ffn_tile_shape(mk(4096, 4096, 64, 2, 32768, has_shared=True)) == "rows"
+    assert native.moe_ffn_tile_shape(mk(16, 4096, 8, 2, 14336)) == "rows"
+    assert native.moe_ffn_tile_shape(mk(8192, 4096, 8, 2, 14336, tiles="columns")) == "columns"
+    assert native.moe_ffn_tile_shape(mk(16, 4096, 8, 2, 14336, tiles="rows")) == "rows"
+    for fuse in ("gather", "combine", "gather+combine"):
+        assert native.moe_ffn_tile_shape(mk(1412, 1024, 32, 8, 512, fuse=fuse)) == "columns"
+        assert native.moe_workspace_bytes(mk(1412, 1024, 32, 8, 512, fuse=fuse, tiles="rows")) == 0
+        assert native.moe_workspace_bytes(mk(64, 64, 4, 2, 128, dtype="f32", fuse=fuse)) == 0
+    assert native.moe_workspace_bytes(mk(1412, 1024, 32, 8, 512, fuse="combine")) > \
+        native.moe_workspace_bytes(mk(1412, 1024, 32, 8, 512))
+    bad = mk(16, 4096, 8, 2, 14336)
+    bad.tiles = 3
+    assert native.lib().moe_ffn_tile_shape(ctypes.byref(bad)) == 0
+    assert native.moe_workspace_bytes(bad) == 0

@@ -144,9 +144,9 @@ def test_dispatch_rejects_bad_ids():
 
 # ------------------------------------------------------------------------- whole layer
 
-def _run_oracle_routing(wl, seed=0):
+def _run_oracle_routing(wl, seed=0, tiles="auto"):
     x, (p,) = I.make_inputs(wl, seed=seed, device="cuda", layers=1)
-    cfg = config_for(wl)
+    cfg = config_for(wl, tiles=tiles)
     C = oracle_capacity(wl)
     ids_ref, g_ref, _ = O.route(x, p["w_router"], p["logit_bias"], wl.k, wl.gate_mode)
     g32 = torch.from_numpy(g_ref.astype(np.float32))
@@ -168,6 +168,67 @@ def test_layer_parity_on_oracle_routing(name):
         bound = 2e-2 * np.max(np.abs(moe_ref)) + 2.0 ** -8 * np.max(np.abs(y_ref))
         assert np.max(np.abs(moe_gpu - moe_ref)) <= bound
     assert_close(out["y"], y_ref, wl.dtype, name)
+
+
+@pytest.mark.parametrize("tiles", ["rows", "columns"])
+@pytest.mark.parametrize("name", ["granite_layer", "switch_phi125", "switch_phi050", "mixtral_T300",
+                                  "mixtral_decode", "shared64_narrow_phi1",
+                                  "shared64_narrow_phi2_T1"])
+def test_both_tile_shapes_on_oracle_routing(name, tiles):
+    """The row-tile and the column-tile FFN kernels, forced on the same inputs and routing,
+    each against the oracle (segments of 1 to a few hundred rows, ragged tails, the shared
+    expert, capacity drops)."""
+    wl, x, p, C, ids_ref, g32, out = _run_oracle_routing(SMALL[name], tiles=tiles)
+    assert out["status"] == 0
+    y_ref, _ = O.moe_layer(x, p, wl.k, wl.gate_mode, C, add_residual=wl.add_residual,
+                           routing=(ids_ref, g32.double().numpy()))
+    if wl.add_residual:
+        moe_ref = y_ref - O.as_f64(x)
+        moe_gpu = out["y"].double().cpu().numpy() - O.as_f64(x)
+        bound = 2e-2 * np.max(np.abs(moe_ref)) + 2.0 ** -8 * np.max(np.abs(y_ref))
+        assert np.max(np.abs(moe_gpu - moe_ref)) <= bound
+    assert_close(out["y"], y_ref, wl.dtype, f"{name} {tiles}")
+
+
+FUSED_CASES = ["tiny_bf16", "granite_layer", "switch_phi050", "mixtral_T300", "mixtral_decode",
+               "shared64_narrow_phi1", "shared64_narrow_dropless", "shared64_narrow_phi2_T1"]
+
+
+@pytest.mark.parametrize("fuse", ["gather", "combine", "gather+combine"])
+@pytest.mark.parametrize("name", FUSED_CASES)
+def test_fused_steps(name, fuse):
+    """moe_forward with the gather fused into the gate/up GEMM and/or the combine fused into
+    the down GEMM's epilogue: bit-identical to the unfused column-tile forward (the same
+    rows are summed in the same order), and within the bar against the oracle."""
+    wl = SMALL[name] if name in SMALL else W["tiny_fp32"].with_(dtype="bf16", d=128, d_ff=128,
+                                                                 add_residual=True)
+    x, (p,) = I.make_inputs(wl, seed=3, device="cuda", layers=1)
+    ref = forward_gpu(config_for(wl, tiles="columns"), x, p)
+    out = forward_gpu(config_for(wl, fuse=fuse), x, p)
+    assert ref["status"] == 0 and out["status"] == 0
+    for key in ("ids", "gates", "demand", "offsets"):
+        assert torch.equal(out[key], ref[key]), key
+    assert torch.equal(out["y"].view(torch.int16), ref["y"].view(torch.int16))
+    C = oracle_capacity(wl)
+    y_ref, info = O.moe_layer(x, p, wl.k, wl.gate_mode, C, add_residual=wl.add_residual)
+    bad, n_near, ok = ids_agree(out["ids"], info["ids"], O.topk_margin(info["logits"], wl.k),
+                                info["logits"], wl.k)
+    assert len(bad) == 0
+    keep = _robust_tokens(info, ok, n_near, C)
+    assert_close(out["y"][torch.from_numpy(keep).cuda()], y_ref[keep], wl.dtype, f"{name} {fuse}")
+
+
+def test_fused_combine_with_every_route_dropped():
+    """Capacity 0: no token has a contribution, so the pack writes y = x (residual) itself."""
+    wl = W["switch_phi100"].with_(T=100, add_residual=True)
+    x, (p,) = I.make_inputs(wl, seed=0, device="cuda", layers=1)
+    for fuse in ("combine", "gather+combine"):
+        out = forward_gpu(config_for(wl, capacity=0, fuse=fuse), x, p)
+        assert out["status"] == 0
+        assert torch.equal(out["y"], x)
+    wl0 = wl.with_(add_residual=False)
+    out = forward_gpu(config_for(wl0, capacity=0, fuse="combine"), x, p)
+    assert out["status"] == 0 and not out["y"].any()
 
 
 @pytest.mark.parametrize("name", list(SMALL))
@@ -253,11 +314,12 @@ def _robust_tokens(info, ok, n_near, C):
 
 # ------------------------------------------------------------------------- full size
 
-@pytest.mark.parametrize("name,sample", [("mixtral_prefill", None), ("mixtral_decode", None),
-                                         ("shared64_T16_dropless", None),
-                                         ("shared64_T4096_dropless", 512),
-                                         ("shared64_T4096_phi1", 64), ("switch_phi050", None)])
-def test_full_size(name, sample):
+@pytest.mark.parametrize("name,sample,tiles", [
+    ("mixtral_prefill", None, ("auto", "columns")), ("mixtral_decode", None, ("auto", "rows")),
+    ("shared64_T16_dropless", None, ("auto", "fused")),
+    ("shared64_T4096_dropless", 512, ("auto", "rows", "fused")),
+    ("shared64_T4096_phi1", 64, ("auto",)), ("switch_phi050", None, ("auto", "rows"))])
+def test_full_size(name, sample, tiles):
     """Full-size layer in the bench's launch configuration.  The oracle routes every token
     and computes the output of every token (sample None) or of a seeded sample of tokens
     (the 64+1 layer at T=4096, whose 52 GB of weights the oracle converts to fp64 expert
@@ -265,8 +327,12 @@ def test_full_size(name, sample):
     capacity, its kept/dropped status cannot be changed by a near-tie token elsewhere."""
     wl = W[name]
     x, (p,) = I.make_inputs(wl, seed=0, device="cuda", layers=1)
-    out = forward_gpu(config_for(wl), x, p)
-    assert out["status"] == 0
+    outs = {t: forward_gpu(config_for(wl, tiles="auto", fuse="gather+combine") if t == "fused"
+                           else config_for(wl, tiles=t), x, p) for t in tiles}
+    out = outs["auto"]
+    for o in outs.values():
+        assert o["status"] == 0
+        assert torch.equal(o["ids"], out["ids"])
     C = oracle_capacity(wl)
     ids_ref, g_ref, z = O.route(x, p["w_router"], p["logit_bias"], wl.k, wl.gate_mode)
     margin = O.topk_margin(z, wl.k)
@@ -287,8 +353,10 @@ def test_full_size(name, sample):
         toks = np.sort(rng.choice(cand, size=min(sample, len(cand)), replace=False))
     y_ref, _ = O.moe_layer(x, p, wl.k, wl.gate_mode, C, add_residual=wl.add_residual,
                            tokens=toks, routing=(ids_ref, g_ref))
-    err, bound = assert_close(out["y"][torch.from_numpy(toks).cuda()], y_ref, wl.dtype, name)
-    print(f"{name}: {len(toks)} of {wl.T} tokens, max|err| {err:.3e} <= {bound:.3e}")
+    for t, o in outs.items():
+        err, bound = assert_close(o["y"][torch.from_numpy(toks).cuda()], y_ref, wl.dtype,
+                                  f"{name} tiles={t}")
+        print(f"{name} tiles={t}: {len(toks)} of {wl.T} tokens, max|err| {err:.3e} <= {bound:.3e}")
 
 
 # ------------------------------------------------------------------------- edge cases
