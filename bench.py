@@ -48,10 +48,10 @@ SPEC_PEAKS = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}
 KERNELS = ["route", "pack", "gemm_gate_up", "gemm_down", "combine"]
 KERNEL_SOURCES = {"route": ["route.cu", "route_sm100.cu", "common.cuh"],
                   "pack": ["dispatch.cu", "reroute.cu", "common.cuh"],
-                  "gemm_gate_up": ["gemm_sm100.cu", "gemm_cols_sm100.cu", "gemm_common.cuh",
-                                   "common.cuh"],
-                  "gemm_down": ["gemm_sm100.cu", "gemm_cols_sm100.cu", "gemm_common.cuh",
-                                "common.cuh"],
+                  "gemm_gate_up": ["gemm_sm100.cu", "gemm_cols_sm100.cu", "gemm_pair_sm100.cu",
+                                   "gemm_common.cuh", "common.cuh"],
+                  "gemm_down": ["gemm_sm100.cu", "gemm_cols_sm100.cu", "gemm_pair_sm100.cu",
+                                "gemm_common.cuh", "common.cuh"],
                   "combine": ["combine.cu", "common.cuh"]}
 
 
@@ -80,7 +80,7 @@ def parse_args(argv=None):
     ap.add_argument("--stats", action="store_true",
                     help="also gather routing statistics: the router's per-tile sums and one "
                          "moe_routing_stats call per layer")
-    ap.add_argument("--tiles", default="auto", choices=["auto", "rows", "columns"],
+    ap.add_argument("--tiles", default="auto", choices=["auto", "rows", "columns", "pairs"],
                     help="expert-FFN tile shape (bf16)")
     ap.add_argument("--fuse", default="none", choices=["none", "gather", "combine", "gather+combine"],
                     help="steps fused into the expert GEMMs (workloads with the reroute policy "

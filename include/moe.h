@@ -89,8 +89,12 @@ typedef enum {
                           * here), column tiles when a fused step is requested            */
   MOE_TILES_ROWS = 1,    /* 128 tokens x 256 output columns per tile: tokens on the MMA's M
                           * side; a segment is padded to a multiple of 128 rows           */
-  MOE_TILES_COLUMNS = 2  /* 128 weight rows x up to 128 tokens per tile: weights on M,
+  MOE_TILES_COLUMNS = 2, /* 128 weight rows x up to 128 tokens per tile: weights on M,
                           * tokens on N; a segment is padded to a multiple of 16 rows     */
+  MOE_TILES_PAIRS = 3    /* column tiles over a pair of SMs (one M = 256 MMA, each SM
+                          * holding half of the token tile); a segment is padded to a
+                          * multiple of 32 rows; needs d and d_ff multiples of 256, else
+                          * row tiles run                                                  */
 } moe_tiles;
 
 /* Steps of moe_forward fused into the expert GEMMs (bit flags; bf16, column tiles, drop

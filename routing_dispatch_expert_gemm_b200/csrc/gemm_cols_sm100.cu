@@ -72,6 +72,8 @@ constexpr int kBoxBytes = kTokBox * BK * 2;
 struct ColMaps {
   CUtensorMap x_routed;   // tokens: packed rows [rmax, d] (gate/up) or H [rows_h, F] (down)
   CUtensorMap x_shared;   // x [T, d]: the shared expert's tokens in the gate/up GEMM
+  CUtensorMap x_routed_full;  // the same two with 128-row boxes: one load for a full
+  CUtensorMap x_shared_full;  // token block (more than 112 tokens)
   CUtensorMap w0_routed;  // W_gate or W_down, experts stacked: [E*N, K]
   CUtensorMap w1_routed;  // W_up [E*N, K]
   CUtensorMap w0_shared;  // shared expert [N, K]
@@ -252,7 +254,10 @@ __global__ void __launch_bounds__(threads_of<GATHER>(), 1)
       const TileCoord tc = decode_tile(s_pre, s_rows, p.nseg, tile);
       const int nbox = (tc.ntok + kTokBox - 1) / kTokBox;
       const bool shared = (tc.s == p.E);
-      const CUtensorMap* mx = (MODE == 0 && shared) ? &maps.x_shared : &maps.x_routed;
+      const bool full_box = nbox * kTokBox > NT - kTokBox;  // 8 boxes: one 128-row load
+      const CUtensorMap* mx =
+          (MODE == 0 && shared) ? (full_box ? &maps.x_shared_full : &maps.x_shared)
+                                : (full_box ? &maps.x_routed_full : &maps.x_routed);
       const int x_row = ((MODE == 0 && shared) ? 0 : s_row0[tc.s]) + tc.tb * NT;
       const CUtensorMap* mw0 = shared ? &maps.w0_shared : &maps.w0_routed;
       const CUtensorMap* mw1 = shared ? &maps.w1_shared : &maps.w1_routed;
@@ -270,9 +275,13 @@ __global__ void __launch_bounds__(threads_of<GATHER>(), 1)
         const int kx = kb * BK;
         tma_load_2d(w_dst, mw0, &full[stage], kx, w_row);
         if (MODE == 0) tma_load_2d(w_dst + W_BYTES, mw1, &full[stage], kx, w_row);
-        if (tma_x)
-          for (int i = 0; i < nbox; ++i)
-            tma_load_2d(x_dst + i * kBoxBytes, mx, &full[stage], kx, x_row + i * kTokBox);
+        if (tma_x) {
+          if (full_box)
+            tma_load_2d(x_dst, mx, &full[stage], kx, x_row);
+          else
+            for (int i = 0; i < nbox; ++i)
+              tma_load_2d(x_dst + i * kBoxBytes, mx, &full[stage], kx, x_row + i * kTokBox);
+        }
         if (++stage == C::STAGES) { stage = 0; phase ^= 1u; wrapped = true; }
       }
     }
@@ -485,14 +494,17 @@ cudaError_t launch_ffn_cols_sm100(const moe_config& c, const FfnArgs& f, cudaStr
   // gate/up + SwiGLU: tokens = packed rows [rmax, d] (x [T, d] for the shared expert)
   ColMaps m1;
   bool ok = encode_2d_box(&m1.x_routed, f.x_packed, c.d, f.rmax, kTokBox) &&
+            encode_2d_box(&m1.x_routed_full, f.x_packed, c.d, f.rmax, NT) &&
             encode_2d_box(&m1.w0_routed, f.w_gate, c.d, static_cast<uint64_t>(c.E) * c.d_ff, BW) &&
             encode_2d_box(&m1.w1_routed, f.w_up, c.d, static_cast<uint64_t>(c.E) * c.d_ff, BW);
   if (c.has_shared)
     ok = ok && encode_2d_box(&m1.x_shared, f.x, c.d, c.T, kTokBox) &&
+         encode_2d_box(&m1.x_shared_full, f.x, c.d, c.T, NT) &&
          encode_2d_box(&m1.w0_shared, f.s_gate, c.d, c.d_ff, BW) &&
          encode_2d_box(&m1.w1_shared, f.s_up, c.d, c.d_ff, BW);
   else
-    m1.x_shared = m1.x_routed, m1.w0_shared = m1.w0_routed, m1.w1_shared = m1.w1_routed;
+    m1.x_shared = m1.x_routed, m1.x_shared_full = m1.x_routed_full, m1.w0_shared = m1.w0_routed,
+    m1.w1_shared = m1.w1_routed;
   if (!ok) return cudaErrorInvalidValue;
   ColParams p1{f.offsets, f.counts, nseg, c.E, c.d, c.d_ff, static_cast<__nv_bfloat16*>(f.h),
                c.d_ff, f.status, kWaitLimitNs, static_cast<const __nv_bfloat16*>(f.x),
@@ -506,12 +518,14 @@ cudaError_t launch_ffn_cols_sm100(const moe_config& c, const FfnArgs& f, cudaStr
   // down: tokens = H [rows_h, F]
   ColMaps m2;
   ok = encode_2d_box(&m2.x_routed, f.h, c.d_ff, rows_h, kTokBox) &&
+       encode_2d_box(&m2.x_routed_full, f.h, c.d_ff, rows_h, NT) &&
        encode_2d_box(&m2.w0_routed, f.w_down, c.d_ff, static_cast<uint64_t>(c.E) * c.d, BW);
   if (c.has_shared)
     ok = ok && encode_2d_box(&m2.w0_shared, f.s_down, c.d_ff, c.d, BW);
   else
     m2.w0_shared = m2.w0_routed;
   m2.x_shared = m2.x_routed;
+  m2.x_shared_full = m2.x_routed_full;
   m2.w1_routed = m2.w0_routed;
   m2.w1_shared = m2.w0_shared;
   if (!ok) return cudaErrorInvalidValue;

@@ -366,12 +366,15 @@ int sm_count() {
 int32_t ffn_tile_shape(const moe_config& c) {
   if (c.fuse != 0) return MOE_TILES_COLUMNS;  // the fused steps live in the column kernel
   if (c.tiles == MOE_TILES_COLUMNS) return MOE_TILES_COLUMNS;
+  if (c.tiles == MOE_TILES_PAIRS && c.d % 256 == 0 && c.d_ff % 256 == 0) return MOE_TILES_PAIRS;
   return MOE_TILES_ROWS;
 }
 
 cudaError_t launch_ffn_sm100(const moe_config& c, const FfnArgs& f, cudaStream_t s,
                              cudaEvent_t mid) {
-  if (ffn_tile_shape(c) == MOE_TILES_COLUMNS) return launch_ffn_cols_sm100(c, f, s, mid);
+  const int32_t shape = ffn_tile_shape(c);
+  if (shape == MOE_TILES_COLUMNS) return launch_ffn_cols_sm100(c, f, s, mid);
+  if (shape == MOE_TILES_PAIRS) return launch_ffn_pair_sm100(c, f, s, mid);
   const int nseg = c.E + (c.has_shared ? 1 : 0);
   const long long rows_h = f.rmax + (c.has_shared ? c.T : 0);
   const long long mt_bound = (rows_h + BM - 1) / BM + nseg;

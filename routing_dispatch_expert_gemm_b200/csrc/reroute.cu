@@ -6,10 +6,10 @@
 //
 // Runs after the arrival-order pack, which has already placed every route that fit and
 // left route_row = -1 on the ones that overflowed.  The reroute is sequential by definition
-// (whether a route finds a free slot depends on every earlier reroute): reroute_walk_kernel
-// walks the overflowed routes in arrival order with one warp, while the other warps of its
-// CTA precompute each route's preference order.  A second, grid-wide kernel copies each
-// moved route's token row and re-evaluates that token's gates by the gate mode over its
+// (whether a route finds a free slot depends on every earlier reroute), but because every
+// expert ranks routes by arrival order the result can be built in phases (see
+// reroute_phase_kernel), one CTA, at most E + 1 phases.  A second, grid-wide kernel copies
+// each moved route's token row and re-evaluates that token's gates by the gate mode over its
 // final experts.
 #include <climits>
 
@@ -69,70 +69,102 @@ __device__ void regate(const int32_t* ids, const float* zkeys, const int32_t* ro
 }
 
 // ---------------------------------------------------------------------------------
-// Placement: the arrival-order walk itself, by one warp, fed by 31 helper warps.
-//  * All 1024 threads first list the overflowed routes in arrival order.
-//  * Helper warps take the listed routes in order and, for each, write into a ring of
-//    chunks in shared memory the token's expert preference order (logit descending, ties
-//    to the lower index: each expert's rank is counted against the whole row of keys) and
-//    the set of experts the token already holds (its ids).
-//  * Warp 0 walks the routes in arrival order: a route takes the first expert of its
-//    preference order that its token does not hold (its ids plus the experts its earlier
-//    routes moved to in this walk) and that has a free slot, found 32 candidates at a time
-//    with a ballot; its slot is the expert's next free one.  With none it stays dropped.
-// Every wait is bounded; on a timeout the kernel records MOE_ERR_TIMEOUT and stops.
+// Phased placement.  Every expert ranks the overflowed routes by arrival order, so the
+// sequential walk is reproduced exactly in phases: each pending route proposes the expert
+// it would take if the experts full at the phase start were the only full ones (its
+// token's best-ranked expert that it does not hold and that is not full, or the next-best
+// one after the token's earlier routes of the same phase); a scan in arrival order counts
+// each expert's proposals and finds the first route whose expert has run out of slots.
+// Every route before it is placed exactly as the walk would place it.  The phase then
+// restarts at that route with at least one more expert full, so there are at most E + 1
+// phases.  Only routes whose proposal became full (and the later routes of the same
+// token) re-choose.
 // ---------------------------------------------------------------------------------
-constexpr int kWalkThreads = 1024;
-constexpr int kWalkWarps = kWalkThreads / 32;
-constexpr int kHelpers = kWalkWarps - 1;  // warps 1 .. 31
-constexpr int kChunk = 32;                // routes per ring chunk
-constexpr int kRing = 4;                  // chunks in the ring
+constexpr int kPhThreads = 1024;
+constexpr int kPhWarps = kPhThreads / 32;
 
-struct WalkArgs {
+struct PhaseArgs {
   const int32_t* ids;      // [T, k]
-  const float* zkeys;      // [T, E] ranking keys (NaN as -inf)
+  const float* zkeys;      // [T, E]
   int32_t* row_token;      // [E * C]
   int32_t* route_row;      // [T, k]
   int32_t* offsets;        // filled-slot counts at offsets[E + 2 + e]
-  int32_t* list;           // [0]: moved routes m, then (token, row) pairs
+  int32_t* list;           // [0]: moved routes n, then (token, row) pairs
   int32_t* ag_r;           // [T * k] overflowed routes (flat index), arrival order
-  int32_t* status;
+  int32_t* ag_c;           // [T * k] proposed / final expert, -1: none
+  int32_t* ag_rank;        // [T * k] rank among the phase's proposals to the same expert
+  int32_t* ag_st;          // [T * k] proposal went stale at the end of the phase
   int T, k, E, C;
-  int64_t limit_ns;
 };
 
-struct RingEntry {
-  uint8_t pref[256];   // experts in the token's preference order
-  uint32_t held[8];    // experts the token holds (its ids)
-  int r;               // flat route index t * k + j; -1: padding past the last route
-  int pad[3];
-};
+__device__ __forceinline__ bool bit_of(const uint32_t (&w)[8], int e) {
+  uint32_t v = 0;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) v = (q == (e >> 5)) ? w[q] : v;
+  return (v >> (e & 31)) & 1u;
+}
+__device__ __forceinline__ void set_bit(uint32_t (&w)[8], int e) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    if (q == (e >> 5)) w[q] |= 1u << (e & 31);
+}
 
-__global__ void __launch_bounds__(kWalkThreads, 1) reroute_walk_kernel(WalkArgs a) {
-  __shared__ int s_cnt[256];
-  __shared__ int s_wtot[kWalkWarps];
-  __shared__ int s_n;
-  __shared__ __align__(16) RingEntry s_ring[kRing][kChunk];
-  __shared__ __align__(8) uint64_t s_full[kRing], s_empty[kRing];
-  __shared__ volatile int s_abort;
+// The expert route i proposes when the phase starts at `pos` and s_full marks full experts.
+__device__ int propose(const PhaseArgs& a, int i, int pos, const uint32_t* s_full) {
+  const int t = a.ag_r[i] / a.k;
+  uint32_t held[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) held[q] = s_full[q];
+  for (int jj = 0; jj < a.k; ++jj) {
+    const int e = a.ids[static_cast<size_t>(t) * a.k + jj];
+    if (e >= 0 && e < a.E) set_bit(held, e);
+  }
+  int m = 0;  // the token's earlier routes still pending in this phase
+  for (int q = i - 1; q >= 0 && a.ag_r[q] / a.k == t; --q) {
+    if (q >= pos) {
+      ++m;
+    } else {
+      const int cq = a.ag_c[q];
+      if (cq >= 0) set_bit(held, cq);
+    }
+  }
+  const float* zrow = a.zkeys + static_cast<size_t>(t) * a.E;
+  int pick = -1;
+  for (int round = 0; round <= m; ++round) {
+    float bv = -INFINITY;
+    int be = -1;
+    for (int e = 0; e < a.E; ++e) {
+      if (bit_of(held, e)) continue;
+      const float v = zrow[e];
+      if (be < 0 || v > bv) { bv = v; be = e; }  // strict: equal keys keep the lower index
+    }
+    if (be < 0) return -1;
+    set_bit(held, be);
+    pick = be;
+  }
+  return pick;
+}
+
+__global__ void __launch_bounds__(kPhThreads, 1) reroute_phase_kernel(PhaseArgs a) {
+  __shared__ int s_cnt[256], s_carry[256], s_inc[256];
+  __shared__ int s_wc[kPhWarps][256];  // per-warp proposal counts per expert, then bases
+  __shared__ uint32_t s_full[8];
+  __shared__ int s_wtot[kPhWarps];
+  __shared__ int s_n, s_istar, s_moved;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = a.E, k = a.k, C = a.C;
   pdl_wait();  // route_row, counts and the keys come from the router and the pack
 
-  for (int e = tid; e < 256; e += kWalkThreads) s_cnt[e] = (e < E) ? a.offsets[E + 2 + e] : C;
-  if (tid == 0) {
-    s_n = 0;
-    s_abort = 0;
-    for (int q = 0; q < kRing; ++q) {
-      mbar_init(&s_full[q], kChunk);  // one arrival per route of the chunk
-      mbar_init(&s_empty[q], 1);      // the walker, once it is done with the chunk
-    }
-    fence_mbar_init();
+  for (int e = tid; e < 256; e += kPhThreads) {
+    s_cnt[e] = (e < E) ? a.offsets[E + 2 + e] : C;
+    s_inc[e] = 0;
   }
+  if (tid == 0) { s_n = 0; s_moved = 0; }
   __syncthreads();
 
-  // 1. overflowed routes, arrival order (block scan of per-warp ballots)
+  // 1. overflowed routes, arrival order
   const int total = a.T * k;  // <= INT_MAX / 2 (validated on the host)
-  for (int base = 0; base < total; base += kWalkThreads) {
+  for (int base = 0; base < total; base += kPhThreads) {
     const int r = base + tid;
     bool flag = false;
     if (r < total) {
@@ -144,7 +176,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1) reroute_walk_kernel(WalkArgs 
     if (lane == 0) s_wtot[warp] = __popc(bal);
     __syncthreads();
     int before = 0, n = 0;
-    for (int w = 0; w < kWalkWarps; ++w) {
+    for (int w = 0; w < kPhWarps; ++w) {
       before += (w < warp) ? s_wtot[w] : 0;
       n += s_wtot[w];
     }
@@ -154,123 +186,101 @@ __global__ void __launch_bounds__(kWalkThreads, 1) reroute_walk_kernel(WalkArgs 
     __syncthreads();
   }
   const int n = s_n;
-  const int nchunks = (n + kChunk - 1) / kChunk;
-  __threadfence_block();  // ag_r (global) written by other threads of this CTA above
-
-  if (warp > 0) {
-    // ------------------------------------------------------------ helpers
-    for (int i = warp - 1; i < nchunks * kChunk; i += kHelpers) {
-      const int c = i / kChunk, slot = c % kRing, pos = i % kChunk;
-      int ok = 1;
-      if (lane == 0)
-        ok = mbar_wait_bounded(&s_empty[slot], ((c / kRing) & 1) ^ 1, &s_abort, a.limit_ns,
-                               a.status);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      RingEntry& en = s_ring[slot][pos];
-      if (i < n) {
-        const int r = a.ag_r[i];
-        const int t = r / k;
-        const float* zrow = a.zkeys + static_cast<size_t>(t) * E;
-        float key[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) key[q] = (q * 32 + lane < E) ? zrow[q * 32 + lane] : -INFINITY;
-        int rank[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) rank[q] = 0;
-        for (int e2 = 0; e2 < E; ++e2) {
-          float z2 = key[0];
-#pragma unroll
-          for (int q = 1; q < 8; ++q) z2 = (q == (e2 >> 5)) ? key[q] : z2;
-          z2 = __shfl_sync(0xffffffffu, z2, e2 & 31);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int e = q * 32 + lane;
-            rank[q] += (z2 > key[q] || (z2 == key[q] && e2 < e)) ? 1 : 0;
-          }
-        }
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (q * 32 + lane < E) en.pref[rank[q]] = static_cast<uint8_t>(q * 32 + lane);
-        int e = (lane < k) ? a.ids[static_cast<size_t>(t) * k + lane] : -1;
-        if (e < 0 || e >= E) e = -1;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-          const uint32_t bit = (e >= 0 && (e >> 5) == w) ? (1u << (e & 31)) : 0u;
-          const uint32_t word = __reduce_or_sync(0xffffffffu, bit);
-          if (lane == 0) en.held[w] = word;
-        }
-        if (lane == 0) en.r = r;
-      } else if (lane == 0) {
-        en.r = -1;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_full[slot]);  // release: the entry is written
+  if (tid < 8) {
+    uint32_t w = 0;
+    for (int b = 0; b < 32; ++b) {
+      const int e = tid * 32 + b;
+      if (e >= E || s_cnt[e] >= C) w |= 1u << b;
     }
-  } else {
-    // ------------------------------------------------------------ the walk (warp 0)
-    int moved = 0;
-    int cur_t = -1;
-    uint32_t extra[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // experts the current token moved to
-    for (int c = 0; c < nchunks; ++c) {
-      const int slot = c % kRing;
-      int ok = 1;
-      if (lane == 0)
-        ok = mbar_wait_bounded(&s_full[slot], (c / kRing) & 1, &s_abort, a.limit_ns, a.status);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) {
-        if (lane == 0) s_abort = 1;
-        break;
-      }
-      for (int pos = 0; pos < kChunk; ++pos) {
-        const RingEntry& en = s_ring[slot][pos];
-        const int r = en.r;
-        if (r < 0) break;
-        const int t = r / k;
-        if (t != cur_t) {
-          cur_t = t;
-#pragma unroll
-          for (int w = 0; w < 8; ++w) extra[w] = 0;
-        }
-        int pick = -1;
-        for (int base = 0; base < E && pick < 0; base += 32) {
-          const int idx = base + lane;
-          int e = -1;
-          bool avail = false;
-          if (idx < E) {
-            e = en.pref[idx];
-            uint32_t hw = en.held[e >> 5];
-#pragma unroll
-            for (int w = 0; w < 8; ++w) hw |= (w == (e >> 5)) ? extra[w] : 0u;
-            avail = !((hw >> (e & 31)) & 1u) && s_cnt[e] < C;
-          }
-          const uint32_t b = __ballot_sync(0xffffffffu, avail);
-          if (b != 0) pick = __shfl_sync(0xffffffffu, e, __ffs(b) - 1);
-        }
-        if (pick >= 0) {
-          if (lane == 0) {
-            const int slot_in_e = s_cnt[pick];
-            s_cnt[pick] = slot_in_e + 1;
-            const int row = pick * C + slot_in_e;
-            a.route_row[r] = row;
-            a.row_token[row] = t;
-            a.list[1 + 2 * moved] = t;
-            a.list[2 + 2 * moved] = row;
-          }
-          ++moved;
-#pragma unroll
-          for (int w = 0; w < 8; ++w)
-            if (w == (pick >> 5)) extra[w] |= 1u << (pick & 31);
-        }
-        __syncwarp();  // lane 0's count update is seen by the next route's checks
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[slot]);  // the chunk's entries may be rewritten
-    }
-    if (lane == 0) a.list[0] = moved;
+    s_full[tid] = w;
   }
   __syncthreads();
-  for (int e = tid; e < E; e += kWalkThreads) a.offsets[E + 2 + e] = s_cnt[e];
+
+  // 2. first proposals (a token's routes are consecutive, each counts its earlier ones)
+  for (int i = tid; i < n; i += kPhThreads) a.ag_c[i] = propose(a, i, 0, s_full);
+  __syncthreads();
+
+  // 3. phases
+  int pos = 0;
+  while (pos < n) {
+    for (int e = tid; e < 256; e += kPhThreads) s_carry[e] = 0;
+    if (tid == 0) s_istar = n;
+    __syncthreads();
+    for (int base = pos; base < n; base += kPhThreads) {
+      for (int x = tid; x < kPhWarps * 256; x += kPhThreads) (&s_wc[0][0])[x] = 0;
+      __syncthreads();
+      const int i = base + tid;
+      const int c = (i < n) ? a.ag_c[i] : -1;
+      const uint32_t peers = __match_any_sync(0xffffffffu, c);
+      const int wrank = __popc(peers & ((1u << lane) - 1u));
+      if (c >= 0 && wrank == 0) s_wc[warp][c] = __popc(peers);
+      __syncthreads();
+      for (int e = tid; e < E; e += kPhThreads) {  // exclusive prefix over warps
+        int run = s_carry[e];
+        for (int w = 0; w < kPhWarps; ++w) {
+          const int v = s_wc[w][e];
+          s_wc[w][e] = run;
+          run += v;
+        }
+        s_carry[e] = run;
+      }
+      __syncthreads();
+      if (c >= 0) {
+        const int rank = s_wc[warp][c] + wrank;
+        a.ag_rank[i] = rank;
+        if (s_cnt[c] + rank >= C) atomicMin(&s_istar, i);
+      }
+      __syncthreads();
+      if (s_istar < n) break;
+    }
+    const int istar = s_istar;
+    // commit the routes before istar
+    for (int i = pos + tid; i < istar; i += kPhThreads) {
+      const int c = a.ag_c[i];
+      if (c < 0) continue;
+      const int r = a.ag_r[i], t = r / k;
+      const int row = c * C + s_cnt[c] + a.ag_rank[i];
+      a.route_row[r] = row;
+      a.row_token[row] = t;
+      const int m = atomicAdd(&s_moved, 1);
+      a.list[1 + 2 * m] = t;
+      a.list[2 + 2 * m] = row;
+      atomicAdd(&s_inc[c], 1);
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kPhThreads) {
+      s_cnt[e] += s_inc[e];
+      s_inc[e] = 0;
+    }
+    __syncthreads();
+    if (tid < 8) {
+      uint32_t w = 0;
+      for (int b = 0; b < 32; ++b) {
+        const int e = tid * 32 + b;
+        if (e >= E || s_cnt[e] >= C) w |= 1u << b;
+      }
+      s_full[tid] = w;
+    }
+    __syncthreads();
+    pos = istar;
+    if (pos >= n) break;
+    // stale proposals: their expert filled up; later routes of the same token follow them
+    for (int i = pos + tid; i < n; i += kPhThreads) {
+      const int c = a.ag_c[i];
+      a.ag_st[i] = (c >= 0 && ((s_full[c >> 5] >> (c & 31)) & 1u)) ? 1 : 0;
+    }
+    __syncthreads();
+    for (int i = pos + tid; i < n; i += kPhThreads) {
+      const int t = a.ag_r[i] / k;
+      bool redo = a.ag_st[i] != 0;
+      for (int q = i - 1; !redo && q >= pos && a.ag_r[q] / k == t; --q) redo = a.ag_st[q] != 0;
+      if (redo) a.ag_c[i] = propose(a, i, pos, s_full);
+    }
+    __syncthreads();
+  }
+  for (int e = tid; e < E; e += kPhThreads) a.offsets[E + 2 + e] = s_cnt[e];
+  if (tid == 0) a.list[0] = s_moved;
+  __syncthreads();
   pdl_trigger();
 }
 
@@ -310,14 +320,14 @@ cudaError_t launch_reroute(const moe_config& c, const void* x, const int32_t* id
                            const float* zkeys, float* gates, void* x_packed, int32_t* row_token,
                            int32_t* route_row, int32_t* offsets, int32_t* scratch, int32_t* status,
                            cudaStream_t s) {
+  (void)status;
   const size_t slots = static_cast<size_t>(c.E) * c.capacity;
   const size_t routes = static_cast<size_t>(c.T) * c.k;
   int32_t* list = scratch;
   int32_t* ag = scratch + 2 * slots + 1;
-  (void)routes;
-  WalkArgs a{ids, zkeys, row_token, route_row, offsets, list, ag, status, c.T, c.k, c.E,
-             c.capacity, kWaitLimitNs};
-  cudaError_t e = launch_pdl(reroute_walk_kernel, dim3(1), dim3(kWalkThreads), 0, s, a);
+  PhaseArgs a{ids, zkeys, row_token, route_row, offsets, list, ag, ag + routes, ag + 2 * routes,
+              ag + 3 * routes, c.T, c.k, c.E, c.capacity};
+  cudaError_t e = launch_pdl(reroute_phase_kernel, dim3(1), dim3(kPhThreads), 0, s, a);
   if (e != cudaSuccess) return e;
   int grid = static_cast<int>((slots + kWarps - 1) / kWarps);
   if (grid > 4 * 148) grid = 4 * 148;

@@ -80,6 +80,13 @@ for _T in (1, 16, 256, 4096):
             bias="normal")
 
 
+# A scaled-down stand-in of the 64+1 layer for profiler captures (16 routed experts of
+# d_ff = 8192 plus the shared one, 3.5 GB of weights; T = 1024 keeps T k / E = 128 rows per
+# expert, the 64+1 layer's segment size at T = 4096).  Not a workload of the pages.
+WORKLOADS["shared16_T1024_F8192"] = _w(
+    "shared16_T1024_F8192", T=1024, d=4096, E=16, k=2, d_ff=8192,
+    gate_mode="softmax_topk_renorm", has_shared=True, router_std=None, bias="normal")
+
 # The Switch-shaped and 64+1 layers with capacity through the padded [E, C, d] buffer and
 # the reroute overflow policy.
 WORKLOADS["switch_phi125_reroute"] = WORKLOADS["switch_phi125"].with_(

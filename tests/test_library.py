@@ -203,6 +203,8 @@ def test_ffn_tile_shape_choice(native):
     assert native.moe_ffn_tile_shape(mk(16, 4096, 8, 2, 14336)) == "rows"
     assert native.moe_ffn_tile_shape(mk(8192, 4096, 8, 2, 14336, tiles="columns")) == "columns"
     assert native.moe_ffn_tile_shape(mk(16, 4096, 8, 2, 14336, tiles="rows")) == "rows"
+    assert native.moe_ffn_tile_shape(mk(16, 4096, 8, 2, 14336, tiles="pairs")) == "pairs"
+    assert native.moe_ffn_tile_shape(mk(16, 768, 4, 1, 2432, tiles="pairs")) == "rows"  # d % 256
     for fuse in ("gather", "combine", "gather+combine"):
         assert native.moe_ffn_tile_shape(mk(1412, 1024, 32, 8, 512, fuse=fuse)) == "columns"
         assert native.moe_workspace_bytes(mk(1412, 1024, 32, 8, 512, fuse=fuse, tiles="rows")) == 0
@@ -210,6 +212,6 @@ def test_ffn_tile_shape_choice(native):
     assert native.moe_workspace_bytes(mk(1412, 1024, 32, 8, 512, fuse="combine")) > \
         native.moe_workspace_bytes(mk(1412, 1024, 32, 8, 512))
     bad = mk(16, 4096, 8, 2, 14336)
-    bad.tiles = 3
+    bad.tiles = 4
     assert native.lib().moe_ffn_tile_shape(ctypes.byref(bad)) == 0
     assert native.moe_workspace_bytes(bad) == 0
