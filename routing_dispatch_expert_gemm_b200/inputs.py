@@ -93,6 +93,11 @@ WORKLOADS["switch_phi125_reroute"] = WORKLOADS["switch_phi125"].with_(
     name="switch_phi125_reroute", layout="padded", overflow="reroute")
 WORKLOADS["shared64_T4096_phi1_reroute"] = WORKLOADS["shared64_T4096_phi1"].with_(
     name="shared64_T4096_phi1_reroute", layout="padded", overflow="reroute")
+# The same routing with d_ff = 1024 (x and the router are drawn before the experts, so the
+# overflow and the reroute work are identical): a stand-in small enough for profiler
+# captures of the reroute kernels.  Not a workload of the pages.
+WORKLOADS["shared64_T4096_phi1_reroute_F1024"] = WORKLOADS["shared64_T4096_phi1_reroute"].with_(
+    name="shared64_T4096_phi1_reroute_F1024", d_ff=1024)
 
 
 def _randn(shape, gen, device, std, dtype):

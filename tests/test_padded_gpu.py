@@ -89,8 +89,8 @@ REROUTE_CASES = {
     "E200_k8_tight": (257, 128, 200, 8, (1, 2), None, "softmax_topk", "bf16"),
     "fp32_router": (200, 64, 6, 2, (1, 1), [2, 1, 0, 0, 0, -1], "softmax_topk_renorm", "f32"),
     "C0": (64, 128, 4, 2, (0, 1), None, "topk_softmax", "bf16"),
-    # more than 12288 routes: the phased placement instead of the window walk
-    "E16_k4_phased_path": (4096, 128, 16, 4, (1, 1), [3, 2, 1] + [0] * 13, "softmax_topk_renorm", "bf16"),
+    # 16384 routes, many overflowing: a long cascade of placement phases
+    "E16_k4_many_phases": (4096, 128, 16, 4, (1, 1), [3, 2, 1] + [0] * 13, "softmax_topk_renorm", "bf16"),
 }
 
 
