@@ -46,8 +46,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # HBM3e bandwidth of one B200.
 SPEC_PEAKS = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}
 KERNELS = ["route", "pack", "gemm_gate_up", "gemm_down", "combine"]
-KERNEL_SOURCES = {"route": ["route.cu", "route_sm100.cu", "common.cuh"],
-                  "pack": ["dispatch.cu", "reroute.cu", "common.cuh"],
+KERNEL_SOURCES = {"route": ["route.cu", "route_sm100.cu", "dispatch_prep.cuh", "common.cuh"],
+                  "pack": ["dispatch.cu", "dispatch_prep.cuh", "reroute.cu", "common.cuh"],
                   "gemm_gate_up": ["gemm_sm100.cu", "gemm_cols_sm100.cu", "gemm_pair_sm100.cu",
                                    "gemm_common.cuh", "common.cuh"],
                   "gemm_down": ["gemm_sm100.cu", "gemm_cols_sm100.cu", "gemm_pair_sm100.cu",
