@@ -94,10 +94,9 @@ Layout layout_of(const moe_config& c) {
   // Routing statistics (only with cfg.stats): per-tile probability sums and fp64 partials.
   L.tile_psum = c.stats ? take(static_cast<size_t>(num_tiles_for(c.T, c.E)) * c.E * 4) : 0;
   L.stats_partial = c.stats ? take(static_cast<size_t>(kStatsMaxBlocks) * c.E * 8) : 0;
-  // Reroute policy (only with it): the router's ranking keys and the list of moved routes.
+  // Reroute policy (only with it): the router's ranking keys and the placement's scratch.
   L.zkeys = reroute(c) ? take(static_cast<size_t>(c.T) * c.E * 4) : 0;
-  L.rlist = reroute(c) ? take((2 * static_cast<size_t>(c.E) * c.capacity + 1 +
-                                4 * static_cast<size_t>(c.T) * c.k) * 4) : 0;
+  L.rlist = reroute(c) ? take(reroute_scratch_bytes(c)) : 0;
   // Fused combine (MOE_FUSE_COMBINE): contributions per token, counters per 32 columns.
   L.need = (c.fuse & MOE_FUSE_COMBINE) ? take(static_cast<size_t>(c.T) * 4) : 0;
   L.counters = (c.fuse & MOE_FUSE_COMBINE) ? take(static_cast<size_t>(c.T) * ((c.d + 31) / 32) * 4)

@@ -63,11 +63,12 @@ cudaError_t launch_routing_stats(const moe_config& c, const float* tile_psum,
                                  double* partial, unsigned int* counter, float* f, float* P,
                                  moe_routing_summary* out, cudaStream_t s);
 
-// Reroute overflow policy on the padded buffer, after the arrival-order pack:
-// places the overflowed routes (one CTA, in phases equivalent to the arrival-order walk),
-// rewrites route_row, row_token, the filled-slot counts (offsets[E+2+e]) and the gates of
-// tokens with a moved route, then copies the moved routes' token rows.
-// scratch: [2 * E * C + 1 + 4 * T * k] int32.
+// Reroute overflow policy on the padded buffer, after the arrival-order pack: ranks each
+// overflowing token's experts (grid-wide), places the overflowed routes (one CTA, in phases
+// equivalent to the arrival-order walk), rewrites route_row, row_token, the filled-slot
+// counts (offsets[E+2+e]) and the gates of tokens with a moved route, then copies the moved
+// routes' token rows.  scratch: reroute_scratch_bytes(c) bytes, 16-byte aligned.
+size_t reroute_scratch_bytes(const moe_config& c);
 cudaError_t launch_reroute(const moe_config& c, const void* x, const int32_t* ids,
                            const float* zkeys, float* gates, void* x_packed, int32_t* row_token,
                            int32_t* route_row, int32_t* offsets, int32_t* scratch,

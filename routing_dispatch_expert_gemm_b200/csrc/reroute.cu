@@ -8,9 +8,9 @@
 // left route_row = -1 on the ones that overflowed.  The reroute is sequential by definition
 // (whether a route finds a free slot depends on every earlier reroute), but because every
 // expert ranks routes by arrival order the result can be built in phases (see
-// reroute_phase_kernel), one CTA, at most E + 1 phases.  A second, grid-wide kernel copies
-// each moved route's token row and re-evaluates that token's gates by the gate mode over its
-// final experts.
+// reroute_phase_kernel), one CTA, at most E + 1 phases.  A grid-wide kernel before it ranks
+// each overflowing token's experts once; one after it copies each moved route's token row
+// and re-evaluates that token's gates by the gate mode over its final experts.
 #include <climits>
 
 #include "common.cuh"
@@ -77,212 +77,471 @@ __device__ void regate(const int32_t* ids, const float* zkeys, const int32_t* ro
 // each expert's proposals and finds the first route whose expert has run out of slots.
 // Every route before it is placed exactly as the walk would place it.  The phase then
 // restarts at that route with at least one more expert full, so there are at most E + 1
-// phases.  Only routes whose proposal became full (and the later routes of the same
-// token) re-choose.
+// phases.  A route proposes again only once its expert is full or an earlier route of its
+// token proposed again.
+//
+// reroute_first_kernel ranks, for every token with an overflowed route, the experts it does
+// not hold (one warp per token), and makes the first proposals; reroute_phase_kernel runs
+// the phases on one CTA, with the pending routes in shared memory when they fit, so that a
+// proposal is a walk along the token's ranking that skips full experts and the token's
+// placed routes.
 // ---------------------------------------------------------------------------------
-constexpr int kPhThreads = 1024;
+constexpr int kPhThreads = 256;
 constexpr int kPhWarps = kPhThreads / 32;
+constexpr int kFirstWarps = 8;      // first kernel: one warp per token
+constexpr int kSmemRoutes = 20480;  // pending-route arrays in shared memory up to T k routes
+constexpr int kNoRoute = -2;        // first-proposal value of a route that did not overflow
 
-struct PhaseArgs {
-  const int32_t* ids;      // [T, k]
-  const float* zkeys;      // [T, E]
-  int32_t* row_token;      // [E * C]
-  int32_t* route_row;      // [T, k]
-  int32_t* offsets;        // filled-slot counts at offsets[E + 2 + e]
-  int32_t* list;           // [0]: moved routes n, then (token, row) pairs
-  int32_t* ag_r;           // [T * k] overflowed routes (flat index), arrival order
-  int32_t* ag_c;           // [T * k] proposed / final expert, -1: none
-  int32_t* ag_rank;        // [T * k] rank among the phase's proposals to the same expert
-  int32_t* ag_st;          // [T * k] proposal went stale at the end of the phase
-  int T, k, E, C;
-};
+__host__ __device__ constexpr int pref_stride(int E) { return (E + 15) & ~15; }
 
-__device__ __forceinline__ bool bit_of(const uint32_t (&w)[8], int e) {
-  uint32_t v = 0;
+// Expert bit sets over NW words (bits at e >= E set where the set means "excluded").
+template <int NW>
+__device__ __forceinline__ void set_bit(uint32_t (&w)[NW], int e) {
 #pragma unroll
-  for (int q = 0; q < 8; ++q) v = (q == (e >> 5)) ? w[q] : v;
-  return (v >> (e & 31)) & 1u;
-}
-__device__ __forceinline__ void set_bit(uint32_t (&w)[8], int e) {
-#pragma unroll
-  for (int q = 0; q < 8; ++q)
+  for (int q = 0; q < NW; ++q)
     if (q == (e >> 5)) w[q] |= 1u << (e & 31);
 }
 
-// The expert route i proposes when the phase starts at `pos` and s_full marks full experts.
-__device__ int propose(const PhaseArgs& a, int i, int pos, const uint32_t* s_full) {
-  const int t = a.ag_r[i] / a.k;
-  uint32_t held[8];
-#pragma unroll
-  for (int q = 0; q < 8; ++q) held[q] = s_full[q];
-  for (int jj = 0; jj < a.k; ++jj) {
-    const int e = a.ids[static_cast<size_t>(t) * a.k + jj];
-    if (e >= 0 && e < a.E) set_bit(held, e);
+struct FirstArgs {
+  const int32_t* ids;      // [T, k]
+  const float* zkeys;      // [T, E]
+  const int32_t* route_row;
+  const int32_t* offsets;  // filled-slot counts at offsets[E + 2 + e]
+  int32_t* prop;           // [T * k] first proposal, -1: none, kNoRoute: did not overflow
+  uint8_t* pref;           // [T, pref_stride(E)] experts the token does not hold, best first
+  int32_t* pref_len;       // [T] entries of the token's list
+  int T, k, E, C;
+};
+
+// One warp per token with an overflowed route.  It ranks the experts the token does not
+// hold (descending key, equal keys to the lower index; NaN keys rank as -inf), stores that
+// order, and makes the first proposals: with nothing placed yet, the token's overflowed
+// routes take, in slot order, the first, second, ... experts of the order that are not full
+// after the arrival-order pass.
+template <int NW>
+__global__ void __launch_bounds__(kFirstWarps * 32) reroute_first_kernel(FirstArgs a) {
+  __shared__ uint32_t s_full[8];
+  __shared__ float s_z[kFirstWarps][256];
+  __shared__ uint32_t s_list[kFirstWarps][64];  // 256 expert bytes per warp
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int k = a.k, E = a.E, Ep = pref_stride(E);
+  pdl_wait();  // route_row and the counts come from the pack, the keys from the router
+  pdl_trigger();
+  if (warp < NW) {
+    const int e = warp * 32 + lane;
+    const bool full = e >= E || a.offsets[E + 2 + e] >= a.C;
+    const uint32_t b = __ballot_sync(0xffffffffu, full);
+    if (lane == 0) s_full[warp] = b;
   }
-  int m = 0;  // the token's earlier routes still pending in this phase
-  for (int q = i - 1; q >= 0 && a.ag_r[q] / a.k == t; --q) {
+  __syncthreads();
+  uint8_t* lst = reinterpret_cast<uint8_t*>(s_list[warp]);
+  for (int t = blockIdx.x * kFirstWarps + warp; t < a.T; t += gridDim.x * kFirstWarps) {
+    const int32_t* row = a.ids + static_cast<size_t>(t) * k;
+    int id = -1;
+    bool ovf = false;
+    if (lane < k) {
+      id = row[lane];
+      ovf = a.route_row[static_cast<size_t>(t) * k + lane] < 0 && route_id_valid(row, lane, id, E);
+    }
+    const uint32_t ovm = __ballot_sync(0xffffffffu, ovf);
+    if (ovm == 0) {
+      if (lane < k) a.prop[static_cast<size_t>(t) * k + lane] = kNoRoute;
+      continue;
+    }
+    uint32_t held[NW];
+    int nheld = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const bool mine = lane < k && id >= 0 && id < E && (id >> 5) == w;
+      held[w] = __reduce_or_sync(0xffffffffu, mine ? 1u << (id & 31) : 0u);
+      nheld += __popc(held[w]);
+    }
+    const float* zrow = a.zkeys + static_cast<size_t>(t) * E;
+    for (int e = lane; e < E; e += 32) {
+      const float v = zrow[e];
+      s_z[warp][e] = (v != v) ? -INFINITY : v;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < NW; ++q) {
+      const int e = lane + 32 * q;
+      if (e >= E || ((held[q] >> lane) & 1u)) continue;
+      const float v = s_z[warp][e];
+      int rank = 0;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+#pragma unroll 8
+        for (int b = 0; b < 32; ++b) {
+          const int e2 = 32 * w + b;
+          if (e2 >= E || ((held[w] >> b) & 1u)) continue;
+          const float u = s_z[warp][e2];
+          rank += (u > v || (u == v && e2 < e)) ? 1 : 0;
+        }
+      }
+      lst[rank] = static_cast<uint8_t>(e);
+    }
+    __syncwarp();
+    const int len = E - nheld;
+    uint32_t* dst = reinterpret_cast<uint32_t*>(a.pref + static_cast<size_t>(t) * Ep);
+    for (int w4 = lane; w4 < Ep / 4; w4 += 32) dst[w4] = s_list[warp][w4];
+    if (lane == 0) a.pref_len[t] = len;
+    // the o-th overflowed route takes the o-th entry whose expert is not full
+    const int ord = ovf ? __popc(ovm & ((1u << lane) - 1u)) : -1;
+    const int last = __popc(ovm) - 1;
+    int pick = -1, before = 0;
+    for (int p0 = 0; p0 < len && before <= last; p0 += 32) {
+      const int p = p0 + lane;
+      const int e = (p < len) ? lst[p] : 0;
+      const bool free_slot = p < len && !((s_full[e >> 5] >> (e & 31)) & 1u);
+      uint32_t b = __ballot_sync(0xffffffffu, free_slot);
+      const int nb = __popc(b);
+      if (ord >= before && ord < before + nb) {
+        for (int r = 0; r < ord - before; ++r) b &= b - 1u;
+        pick = lst[p0 + __ffs(b) - 1];
+      }
+      before += nb;
+    }
+    if (lane < k) a.prop[static_cast<size_t>(t) * k + lane] = ovf ? pick : kNoRoute;
+    __syncwarp();
+  }
+}
+
+struct PhaseArgs {
+  const float* zkeys;      // [T, E]
+  const int32_t* prop;     // [T * k] first proposals
+  const uint8_t* pref;     // [T, pref_stride(E)]
+  const int32_t* pref_len; // [T]
+  int32_t* row_token;      // [E * C]
+  int32_t* route_row;      // [T, k]
+  int32_t* offsets;        // filled-slot counts at offsets[E + 2 + e]
+  int32_t* list;           // [0]: n overflowed routes, then (token, row) each; token -1: dropped
+  int32_t* g_r;            // [T * k] pending-route arrays when they are not in shared memory
+  int32_t* g_c;
+  uint8_t* g_dirty;
+  int T, k, E, C;
+  int in_smem;             // 1: the pending-route arrays live in dynamic shared memory
+};
+
+// The first chunks of a token's ranking, requested together.
+template <int NW>
+struct Ranking {
+  static constexpr int kChunks = (NW * 2 < 4) ? NW * 2 : 4;  // <= the row's pref_stride(E) / 16
+  uint4 ck[kChunks];
+  int len;
+};
+
+template <int NW>
+__device__ __forceinline__ void load_ranking(const PhaseArgs& a, int t, Ranking<NW>& r) {
+  const uint4* row =
+      reinterpret_cast<const uint4*>(a.pref + static_cast<size_t>(t) * pref_stride(a.E));
+  r.len = a.pref_len[t];
+#pragma unroll
+  for (int c = 0; c < Ranking<NW>::kChunks; ++c)
+    r.ck[c] = (c * 16 < a.E) ? row[c] : make_uint4(0, 0, 0, 0);
+}
+
+// Route i proposes again, with the experts in s_full full and routes before `pos` placed:
+// the (m+1)-th entry of its token's ranking that is neither full nor taken by one of the
+// token's placed routes, m being the token's earlier routes still pending.  Pending routes
+// are stored as token << 5 | slot.  The excluded experts are one 64-bit register for
+// E <= 64, else the calling thread's column of words in shared memory (word w at
+// ex[w * kPhThreads]).
+template <int NW>
+__device__ __forceinline__ int propose(const PhaseArgs& a, const int* ag_r, const int* ag_c, int i,
+                                       int pos, const uint32_t* s_full, uint32_t* ex) {
+  const int t = ag_r[i] >> 5;
+  Ranking<NW> rk;
+  load_ranking(a, t, rk);
+  uint64_t ex64 = 0;
+  if constexpr (NW <= 2) {
+    ex64 = s_full[0] | (static_cast<uint64_t>(NW == 2 ? s_full[1] : 0xffffffffu) << 32);
+  } else {
+#pragma unroll
+    for (int w = 0; w < NW; ++w) ex[w * kPhThreads] = s_full[w];
+  }
+  int m = 0;
+  for (int q = i - 1; q >= 0 && (ag_r[q] >> 5) == t; --q) {
     if (q >= pos) {
       ++m;
     } else {
-      const int cq = a.ag_c[q];
-      if (cq >= 0) set_bit(held, cq);
+      const int cq = ag_c[q];
+      if (cq >= 0) {
+        if constexpr (NW <= 2) ex64 |= 1ull << cq;
+        else ex[(cq >> 5) * kPhThreads] |= 1u << (cq & 31);
+      }
     }
   }
-  const float* zrow = a.zkeys + static_cast<size_t>(t) * a.E;
-  int pick = -1;
-  for (int round = 0; round <= m; ++round) {
-    float bv = -INFINITY;
-    int be = -1;
-    for (int e = 0; e < a.E; ++e) {
-      if (bit_of(held, e)) continue;
-      const float v = zrow[e];
-      if (be < 0 || v > bv) { bv = v; be = e; }  // strict: equal keys keep the lower index
+  const int len = rk.len;
+  for (int p0 = 0; p0 < len; p0 += 16) {
+    const int c = p0 >> 4;
+    uint4 cur = rk.ck[0];
+    bool have = false;
+#pragma unroll
+    for (int cc = 0; cc < Ranking<NW>::kChunks; ++cc)
+      if (c == cc) { cur = rk.ck[cc]; have = true; }
+    if (!have)
+      cur = reinterpret_cast<const uint4*>(a.pref + static_cast<size_t>(t) * pref_stride(a.E))[c];
+    const uint32_t w4[4] = {cur.x, cur.y, cur.z, cur.w};
+    // all sixteen tests at once (entries past len are masked off afterwards; the index is
+    // clamped so that their bytes stay inside the excluded set's words)
+    uint32_t avail = 0;
+#pragma unroll
+    for (int b = 0; b < 16; ++b) {
+      const int e = ((w4[b >> 2] >> (8 * (b & 3))) & 0xff) & (32 * NW - 1);
+      uint32_t bit;
+      if constexpr (NW <= 2) bit = static_cast<uint32_t>(~ex64 >> e) & 1u;
+      else bit = (~ex[(e >> 5) * kPhThreads] >> (e & 31)) & 1u;
+      avail |= bit << b;
     }
-    if (be < 0) return -1;
-    set_bit(held, be);
-    pick = be;
+    if (len - p0 < 16) avail &= (1u << (len - p0)) - 1u;
+    const int na = __popc(avail);
+    if (m < na) {
+      for (int r = 0; r < m; ++r) avail &= avail - 1u;
+      const int b = __ffs(avail) - 1;
+      const uint32_t w = (b < 4) ? cur.x : (b < 8) ? cur.y : (b < 12) ? cur.z : cur.w;
+      return (w >> (8 * (b & 3))) & 0xff;
+    }
+    m -= na;
   }
-  return pick;
+  return -1;
 }
 
+// The ranking of the token of pending route i into this SM's L1, ahead of a proposal.
+__device__ __forceinline__ void prefetch_ranking(const PhaseArgs& a, int t) {
+  const uint8_t* row = a.pref + static_cast<size_t>(t) * pref_stride(a.E);
+  for (int off = 0; off < pref_stride(a.E); off += 128)
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(row + off));
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(a.pref_len + t));
+}
+
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+  for (int s = 1; s < 32; s <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, v, s);
+    if (lane >= s) v += o;
+  }
+  return v;
+}
+
+template <int NW, bool SMEM>
 __global__ void __launch_bounds__(kPhThreads, 1) reroute_phase_kernel(PhaseArgs a) {
-  __shared__ int s_cnt[256], s_carry[256], s_inc[256];
-  __shared__ int s_wc[kPhWarps][256];  // per-warp proposal counts per expert, then bases
-  __shared__ uint32_t s_full[8];
-  __shared__ int s_wtot[kPhWarps];
-  __shared__ int s_n, s_istar, s_moved;
+  extern __shared__ int s_dyn[];
+  __shared__ int s_wc[kPhWarps][257];  // per-warp proposal counts per expert in the block
+  __shared__ int s_cnt[2][256];         // filled slots: this phase's, and the next phase's
+  __shared__ uint32_t s_full[2][8];     // full experts (and e >= E), likewise
+  __shared__ int s_carry[256];          // proposals per expert in the phase's earlier blocks
+  __shared__ int s_wtot[2][kPhWarps];
+  __shared__ int s_istar[2];
+  __shared__ uint32_t s_ex[NW * kPhThreads];  // per-thread excluded-expert words (propose)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t lt = (1u << lane) - 1u;
   const int E = a.E, k = a.k, C = a.C;
-  pdl_wait();  // route_row, counts and the keys come from the router and the pack
-
-  for (int e = tid; e < 256; e += kPhThreads) {
-    s_cnt[e] = (e < E) ? a.offsets[E + 2 + e] : C;
-    s_inc[e] = 0;
-  }
-  if (tid == 0) { s_n = 0; s_moved = 0; }
-  __syncthreads();
-
-  // 1. overflowed routes, arrival order
   const int total = a.T * k;  // <= INT_MAX / 2 (validated on the host)
-  for (int base = 0; base < total; base += kPhThreads) {
-    const int r = base + tid;
-    bool flag = false;
-    if (r < total) {
-      const int t = r / k, j = r - t * k;
-      const int32_t* row = a.ids + static_cast<size_t>(t) * k;
-      flag = a.route_row[r] < 0 && route_id_valid(row, j, row[j], E);
-    }
-    const uint32_t bal = __ballot_sync(0xffffffffu, flag);
-    if (lane == 0) s_wtot[warp] = __popc(bal);
-    __syncthreads();
-    int before = 0, n = 0;
-    for (int w = 0; w < kPhWarps; ++w) {
-      before += (w < warp) ? s_wtot[w] : 0;
-      n += s_wtot[w];
-    }
-    if (flag) a.ag_r[s_n + before + __popc(bal & ((1u << lane) - 1u))] = r;
-    __syncthreads();
-    if (tid == 0) s_n += n;
-    __syncthreads();
-  }
-  const int n = s_n;
-  if (tid < 8) {
-    uint32_t w = 0;
-    for (int b = 0; b < 32; ++b) {
-      const int e = tid * 32 + b;
-      if (e >= E || s_cnt[e] >= C) w |= 1u << b;
-    }
-    s_full[tid] = w;
-  }
-  __syncthreads();
+  // pending routes in arrival order: token << 5 | slot, proposed / final expert (-1: none),
+  // and a flag set when an earlier route of the same token proposed again
+  int* ag_r = SMEM ? s_dyn : a.g_r;
+  int* ag_c = SMEM ? s_dyn + total : a.g_c;
+  uint8_t* dirty = SMEM ? reinterpret_cast<uint8_t*>(s_dyn + 2 * total) : a.g_dirty;
+  pdl_wait();
 
-  // 2. first proposals (a token's routes are consecutive, each counts its earlier ones)
-  for (int i = tid; i < n; i += kPhThreads) a.ag_c[i] = propose(a, i, 0, s_full);
-  __syncthreads();
+  for (int x = tid; x < kPhWarps * 257; x += kPhThreads) (&s_wc[0][0])[x] = 0;
+  for (int e = tid; e < 256; e += kPhThreads) {  // a warp covers one 32-expert word
+    const int cnt = (e < E) ? a.offsets[E + 2 + e] : C;
+    s_cnt[0][e] = cnt;
+    const uint32_t b = __ballot_sync(0xffffffffu, e >= E || cnt >= C);
+    if (lane == 0) s_full[0][e >> 5] = b;
+  }
 
-  // 3. phases
-  int pos = 0;
-  while (pos < n) {
-    for (int e = tid; e < 256; e += kPhThreads) s_carry[e] = 0;
-    if (tid == 0) s_istar = n;
+  // 1. overflowed routes in arrival order, sixteen consecutive routes per thread
+  int n = 0;
+  for (int base = 0, pass = 0; base < total; base += 16 * kPhThreads, ++pass) {
+    const int r0 = base + 16 * tid;
+    int v[16];
+    if (r0 + 16 <= total) {  // prop is 16-byte aligned
+      const int4* p4 = reinterpret_cast<const int4*>(a.prop + r0);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int4 q = p4[u];
+        v[4 * u] = q.x; v[4 * u + 1] = q.y; v[4 * u + 2] = q.z; v[4 * u + 3] = q.w;
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < 16; ++u) v[u] = (r0 + u < total) ? a.prop[r0 + u] : kNoRoute;
+    }
+    uint32_t bits = 0;
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+      if (v[u] != kNoRoute) bits |= 1u << u;
+    const int cnt = __popc(bits);
+    const int incl = warp_incl_scan(cnt, lane);
+    if (lane == 31) s_wtot[pass & 1][warp] = incl;
     __syncthreads();
-    for (int base = pos; base < n; base += kPhThreads) {
-      for (int x = tid; x < kPhWarps * 256; x += kPhThreads) (&s_wc[0][0])[x] = 0;
-      __syncthreads();
-      const int i = base + tid;
-      const int c = (i < n) ? a.ag_c[i] : -1;
-      const uint32_t peers = __match_any_sync(0xffffffffu, c);
-      const int wrank = __popc(peers & ((1u << lane) - 1u));
-      if (c >= 0 && wrank == 0) s_wc[warp][c] = __popc(peers);
-      __syncthreads();
-      for (int e = tid; e < E; e += kPhThreads) {  // exclusive prefix over warps
-        int run = s_carry[e];
-        for (int w = 0; w < kPhWarps; ++w) {
-          const int v = s_wc[w][e];
-          s_wc[w][e] = run;
-          run += v;
+    const int wv = (lane < kPhWarps) ? s_wtot[pass & 1][lane] : 0;
+    const int wincl = warp_incl_scan(wv, lane);
+    const int wexcl = __shfl_sync(0xffffffffu, wincl - wv, warp);
+    const int ptot = __shfl_sync(0xffffffffu, wincl, 31);
+    int out = n + wexcl + incl - cnt;
+    if (bits != 0) {
+      int t = r0 / k, j = r0 - t * k;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        if ((bits >> u) & 1u) {
+          ag_r[out] = (t << 5) | j;
+          ag_c[out] = v[u];
+          dirty[out] = 0;
+          ++out;
         }
-        s_carry[e] = run;
+        if (++j == k) { j = 0; ++t; }
       }
-      __syncthreads();
-      if (c >= 0) {
-        const int rank = s_wc[warp][c] + wrank;
-        a.ag_rank[i] = rank;
-        if (s_cnt[c] + rank >= C) atomicMin(&s_istar, i);
-      }
-      __syncthreads();
-      if (s_istar < n) break;
     }
-    const int istar = s_istar;
-    // commit the routes before istar
-    for (int i = pos + tid; i < istar; i += kPhThreads) {
-      const int c = a.ag_c[i];
-      if (c < 0) continue;
-      const int r = a.ag_r[i], t = r / k;
-      const int row = c * C + s_cnt[c] + a.ag_rank[i];
-      a.route_row[r] = row;
-      a.row_token[row] = t;
-      const int m = atomicAdd(&s_moved, 1);
-      a.list[1 + 2 * m] = t;
-      a.list[2 + 2 * m] = row;
-      atomicAdd(&s_inc[c], 1);
-    }
-    __syncthreads();
-    for (int e = tid; e < E; e += kPhThreads) {
-      s_cnt[e] += s_inc[e];
-      s_inc[e] = 0;
-    }
-    __syncthreads();
-    if (tid < 8) {
-      uint32_t w = 0;
-      for (int b = 0; b < 32; ++b) {
-        const int e = tid * 32 + b;
-        if (e >= E || s_cnt[e] >= C) w |= 1u << b;
-      }
-      s_full[tid] = w;
-    }
-    __syncthreads();
-    pos = istar;
-    if (pos >= n) break;
-    // stale proposals: their expert filled up; later routes of the same token follow them
-    for (int i = pos + tid; i < n; i += kPhThreads) {
-      const int c = a.ag_c[i];
-      a.ag_st[i] = (c >= 0 && ((s_full[c >> 5] >> (c & 31)) & 1u)) ? 1 : 0;
-    }
-    __syncthreads();
-    for (int i = pos + tid; i < n; i += kPhThreads) {
-      const int t = a.ag_r[i] / k;
-      bool redo = a.ag_st[i] != 0;
-      for (int q = i - 1; !redo && q >= pos && a.ag_r[q] / k == t; --q) redo = a.ag_st[q] != 0;
-      if (redo) a.ag_c[i] = propose(a, i, pos, s_full);
-    }
-    __syncthreads();
+    n += ptot;
   }
-  for (int e = tid; e < E; e += kPhThreads) a.offsets[E + 2 + e] = s_cnt[e];
-  if (tid == 0) a.list[0] = s_moved;
+  if (tid == 0) s_istar[0] = n;
+  __syncthreads();
+  if (tid < n) prefetch_ranking(a, ag_r[tid] >> 5);
+
+  // 2. phases.  Each scan block first brings its routes' proposals up to date: a route
+  //    proposes again when its expert is full, when an earlier pending route of its token in
+  //    the block does, or when it is marked dirty (a route of its token in an earlier block
+  //    proposed again).  Routes past the scanned blocks are brought up to date when a later
+  //    phase reaches them: a proposal whose expert is not full stays what it would be.
+  //    Placements of a phase go to the next phase's counts and full set, so that one
+  //    barrier ends a phase.
+  int pos = 0, cur = 0;
+  while (pos < n) {
+    const int nxt = cur ^ 1;
+    int istar = n;
+    for (int base = pos; base < n; base += kPhThreads) {
+      const int i = base + tid;
+      if (base == pos) {  // a phase's first block: start the next phase's state from this one's
+        for (int e = tid; e < 256; e += kPhThreads) {
+          s_cnt[nxt][e] = s_cnt[cur][e];
+          s_carry[e] = 0;
+        }
+        if (tid < 8) s_full[nxt][tid] = s_full[cur][tid];
+        if (tid == 0) s_istar[nxt] = n;
+      }
+      const uint32_t* full = s_full[cur];
+      // (each thread judges its token's earlier routes in the block itself; the new
+      // proposals and flags are stored only after the next barrier)
+      int c = -1, tr = 0;
+      bool again = false;
+      if (i < n) {
+        c = ag_c[i];
+        tr = ag_r[i];
+        again = dirty[i] != 0 || (c >= 0 && ((full[c >> 5] >> (c & 31)) & 1u));
+        const int t = tr >> 5;
+        for (int q = i - 1; !again && q >= base && (ag_r[q] >> 5) == t; --q) {
+          const int cq = ag_c[q];
+          again = dirty[q] != 0 || (cq >= 0 && ((full[cq >> 5] >> (cq & 31)) & 1u));
+        }
+      }
+      if (again) c = propose<NW>(a, ag_r, ag_c, i, pos, full, s_ex + tid);
+      // scan in arrival order; place every route before the first one whose expert has no
+      // slot left for it.  A route's rank among the block's proposals to its expert is its
+      // rank in its warp plus the earlier warps' counts.
+      const uint32_t peers = __match_any_sync(0xffffffffu, c);
+      const int wrank = __popc(peers & lt);
+      const bool lead = c >= 0 && wrank == 0;
+      __syncwarp();  // this warp's counts of the previous block are cleared
+      if (lead) s_wc[warp][c] = __popc(peers);
+      __syncthreads();
+      if (again) {
+        ag_c[i] = c;
+        dirty[i] = 0;
+        const int t = tr >> 5;
+        for (int q = i + 1; q < n && (ag_r[q] >> 5) == t; ++q)
+          if (q >= base + kPhThreads) dirty[q] = 1;
+      }
+      int rank = 0;
+      if (c >= 0) {
+        rank = s_carry[c] + wrank;
+#pragma unroll
+        for (int w = 0; w < kPhWarps; ++w)
+          if (w < warp) rank += s_wc[w][c];
+      }
+      const uint32_t over = __ballot_sync(0xffffffffu, c >= 0 && s_cnt[cur][c] + rank >= C);
+      if (over != 0 && lane == __ffs(over) - 1) atomicMin(&s_istar[cur], i);  // warp's first
+      __syncthreads();
+      istar = s_istar[cur];
+      {  // the route this thread handles in the next block: its ranking into L1
+        const int nx = ((istar < n) ? istar : base + kPhThreads) + tid;
+        if (nx < n) prefetch_ranking(a, ag_r[nx] >> 5);
+      }
+      if (lead) {
+        s_wc[warp][c] = 0;
+        if (istar == n) atomicAdd(&s_carry[c], __popc(peers));
+      }
+      const bool placed = c >= 0 && i < istar;
+      const uint32_t grp = peers & __ballot_sync(0xffffffffu, placed);
+      if (i < istar && i < n) {  // placed, or dropped for good when no expert is left
+        const int t = tr >> 5;
+        if (c >= 0) {
+          const int slot = s_cnt[cur][c] + rank;
+          const int row = c * C + slot;
+          a.route_row[static_cast<size_t>(t) * k + (tr & 31)] = row;
+          a.row_token[row] = t;
+          a.list[1 + 2 * i] = t;
+          a.list[2 + 2 * i] = row;
+          // the group's last placed lane holds its highest slot
+          if ((grp >> lane) == 1u) atomicMax(&s_cnt[nxt][c], slot + 1);
+          if (slot + 1 == C) atomicOr(&s_full[nxt][c >> 5], 1u << (c & 31));
+        } else {
+          a.list[1 + 2 * i] = -1;
+        }
+      }
+      if (istar < n) break;
+    }
+    __syncthreads();
+    cur = nxt;
+    pos = istar;
+  }
+  for (int e = tid; e < E; e += kPhThreads) a.offsets[E + 2 + e] = s_cnt[cur][e];
+  if (tid == 0) a.list[0] = n;
   __syncthreads();
   pdl_trigger();
 }
+
+constexpr int kRouteSmemBytes = 2 * sizeof(int) + 1;  // ag_r, ag_c, dirty
+
+template <int NW>
+cudaError_t launch_placement(const FirstArgs& fa, const PhaseArgs& pa, cudaStream_t s) {
+  static DeviceOnce once;
+  cudaError_t e = once.run([] {
+    return cudaFuncSetAttribute(reroute_phase_kernel<NW, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kSmemRoutes * kRouteSmemBytes);
+  });
+  if (e != cudaSuccess) return e;
+  int grid = (fa.T + kFirstWarps - 1) / kFirstWarps;
+  if (grid > 8 * 148) grid = 8 * 148;
+  e = launch_pdl(reroute_first_kernel<NW>, dim3(grid), dim3(kFirstWarps * 32), 0, s, fa);
+  if (e != cudaSuccess) return e;
+  if (pa.in_smem)
+    return launch_pdl(reroute_phase_kernel<NW, true>, dim3(1), dim3(kPhThreads),
+                      static_cast<size_t>(pa.T) * pa.k * kRouteSmemBytes, s, pa);
+  return launch_pdl(reroute_phase_kernel<NW, false>, dim3(1), dim3(kPhThreads), 0, s, pa);
+}
+
+// Scratch: the moved-route list (2 T k + 1, padded to 4), first proposals and the pending-
+// route arrays (4 T k), the ranking lengths (T), then the rankings (T pref_stride(E) bytes).
+size_t list_ints(const moe_config& c) {  // rounded up so that what follows is 16-byte aligned
+  return (2 * static_cast<size_t>(c.T) * c.k + 1 + 3) & ~static_cast<size_t>(3);
+}
+size_t scratch_ints(const moe_config& c) {
+  return list_ints(c) + 4 * static_cast<size_t>(c.T) * c.k + static_cast<size_t>(c.T);
+}
+size_t pref_offset(const moe_config& c) {
+  return (scratch_ints(c) * 4 + 15) & ~static_cast<size_t>(15);
+}
+
+}  // namespace
+
+size_t reroute_scratch_bytes(const moe_config& c) {
+  return pref_offset(c) + static_cast<size_t>(c.T) * pref_stride(c.E);
+}
+
+namespace {
 
 struct CopyArgs {
   const void* x;
@@ -295,8 +554,9 @@ struct CopyArgs {
   int d, k, E, C, gate_mode;
 };
 
-// One warp per moved route: copy x[t] to its new row of the padded buffer and re-evaluate
-// token t's gates (a token with two moved routes is evaluated twice, to the same values).
+// One warp per overflowed route that moved: copy x[t] to its new row of the padded buffer
+// and re-evaluate token t's gates (a token with two moved routes is evaluated twice, to the
+// same values).
 template <typename T>
 __global__ void __launch_bounds__(kThreads) reroute_copy_kernel(CopyArgs a) {
   constexpr int VEC = Vec<T>::N;
@@ -307,6 +567,7 @@ __global__ void __launch_bounds__(kThreads) reroute_copy_kernel(CopyArgs a) {
   const int nvec = a.d / VEC;
   for (int i = blockIdx.x * kWarps + warp; i < n; i += gridDim.x * kWarps) {
     const int t = a.list[1 + 2 * i], row = a.list[2 + 2 * i];
+    if (t < 0) continue;  // no expert had a slot left
     const T* src = static_cast<const T*>(a.x) + static_cast<size_t>(t) * a.d;
     T* dst = static_cast<T*>(a.x_packed) + static_cast<size_t>(row) * a.d;
     for (int v = lane; v < nvec; v += 32) st_vec(dst + v * VEC, ld_vec(src + v * VEC));
@@ -324,10 +585,19 @@ cudaError_t launch_reroute(const moe_config& c, const void* x, const int32_t* id
   const size_t slots = static_cast<size_t>(c.E) * c.capacity;
   const size_t routes = static_cast<size_t>(c.T) * c.k;
   int32_t* list = scratch;
-  int32_t* ag = scratch + 2 * slots + 1;
-  PhaseArgs a{ids, zkeys, row_token, route_row, offsets, list, ag, ag + routes, ag + 2 * routes,
-              ag + 3 * routes, c.T, c.k, c.E, c.capacity};
-  cudaError_t e = launch_pdl(reroute_phase_kernel, dim3(1), dim3(kPhThreads), 0, s, a);
+  int32_t* prop = scratch + list_ints(c);
+  int32_t* pref_len = prop + 4 * routes;
+  uint8_t* pref = reinterpret_cast<uint8_t*>(scratch) + pref_offset(c);
+  const FirstArgs fa{ids,  zkeys,    route_row, offsets, prop,      pref,
+                     pref_len, c.T, c.k,       c.E,     c.capacity};
+  const PhaseArgs pa{zkeys, prop, pref, pref_len, row_token, route_row, offsets, list,
+                     prop + routes, prop + 2 * routes,
+                     reinterpret_cast<uint8_t*>(prop + 3 * routes), c.T, c.k, c.E, c.capacity,
+                     routes <= static_cast<size_t>(kSmemRoutes) ? 1 : 0};
+  cudaError_t e = c.E <= 32   ? launch_placement<1>(fa, pa, s)
+                  : c.E <= 64  ? launch_placement<2>(fa, pa, s)
+                  : c.E <= 128 ? launch_placement<4>(fa, pa, s)
+                               : launch_placement<8>(fa, pa, s);
   if (e != cudaSuccess) return e;
   int grid = static_cast<int>((slots + kWarps - 1) / kWarps);
   if (grid > 4 * 148) grid = 4 * 148;
