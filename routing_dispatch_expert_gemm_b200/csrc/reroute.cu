@@ -92,6 +92,16 @@ constexpr int kFirstWarps = 8;      // first kernel: one warp per token
 constexpr int kSmemRoutes = 20480;  // pending-route arrays in shared memory up to T k routes
 constexpr int kNoRoute = -2;        // first-proposal value of a route that did not overflow
 
+// A proposal with the position in the token's ranking that the next walk starts from
+// (expert 0xffff: none; the position is then the ranking's length).
+__host__ __device__ constexpr int prop_pack(int expert, int at) {
+  return (at << 16) | (expert & 0xffff);
+}
+__host__ __device__ constexpr int prop_expert(int v) {
+  return ((v & 0xffff) == 0xffff) ? -1 : (v & 0xffff);
+}
+__host__ __device__ constexpr int prop_at(int v) { return v >> 16; }
+
 __host__ __device__ constexpr int pref_stride(int E) { return (E + 15) & ~15; }
 
 // Expert bit sets over NW words (bits at e >= E set where the set means "excluded").
@@ -107,7 +117,7 @@ struct FirstArgs {
   const float* zkeys;      // [T, E]
   const int32_t* route_row;
   const int32_t* offsets;  // filled-slot counts at offsets[E + 2 + e]
-  int32_t* prop;           // [T * k] first proposal, -1: none, kNoRoute: did not overflow
+  int32_t* prop;           // [T * k] first proposal (prop_pack), kNoRoute: did not overflow
   uint8_t* pref;           // [T, pref_stride(E)] experts the token does not hold, best first
   int32_t* pref_len;       // [T] entries of the token's list
   int T, k, E, C;
@@ -188,7 +198,7 @@ __global__ void __launch_bounds__(kFirstWarps * 32) reroute_first_kernel(FirstAr
     // the o-th overflowed route takes the o-th entry whose expert is not full
     const int ord = ovf ? __popc(ovm & ((1u << lane) - 1u)) : -1;
     const int last = __popc(ovm) - 1;
-    int pick = -1, before = 0;
+    int pick = prop_pack(-1, len), before = 0;
     for (int p0 = 0; p0 < len && before <= last; p0 += 32) {
       const int p = p0 + lane;
       const int e = (p < len) ? lst[p] : 0;
@@ -197,7 +207,8 @@ __global__ void __launch_bounds__(kFirstWarps * 32) reroute_first_kernel(FirstAr
       const int nb = __popc(b);
       if (ord >= before && ord < before + nb) {
         for (int r = 0; r < ord - before; ++r) b &= b - 1u;
-        pick = lst[p0 + __ffs(b) - 1];
+        const int at = p0 + __ffs(b) - 1;
+        pick = prop_pack(lst[at], at);
       }
       before += nb;
     }
@@ -218,6 +229,7 @@ struct PhaseArgs {
   int32_t* g_r;            // [T * k] pending-route arrays when they are not in shared memory
   int32_t* g_c;
   uint8_t* g_dirty;
+  uint8_t* g_at;
   int T, k, E, C;
   int in_smem;             // 1: the pending-route arrays live in dynamic shared memory
 };
@@ -243,12 +255,14 @@ __device__ __forceinline__ void load_ranking(const PhaseArgs& a, int t, Ranking<
 // Route i proposes again, with the experts in s_full full and routes before `pos` placed:
 // the (m+1)-th entry of its token's ranking that is neither full nor taken by one of the
 // token's placed routes, m being the token's earlier routes still pending.  Pending routes
-// are stored as token << 5 | slot.  The excluded experts are one 64-bit register for
-// E <= 64, else the calling thread's column of words in shared memory (word w at
-// ex[w * kPhThreads]).
+// are stored as token << 5 | slot.  With m = 0 the walk resumes at the route's last
+// position `at`: every entry before it was full, or taken by the token's placed or earlier
+// routes, and stays so.  The excluded experts are one 64-bit register for E <= 64, else the
+// calling thread's column of words in shared memory (word w at ex[w * kPhThreads]).
+// Returns the expert (-1: none) and updates `at`.
 template <int NW>
 __device__ __forceinline__ int propose(const PhaseArgs& a, const int* ag_r, const int* ag_c, int i,
-                                       int pos, const uint32_t* s_full, uint32_t* ex) {
+                                       int pos, const uint32_t* s_full, uint32_t* ex, int& at) {
   const int t = ag_r[i] >> 5;
   Ranking<NW> rk;
   load_ranking(a, t, rk);
@@ -272,7 +286,8 @@ __device__ __forceinline__ int propose(const PhaseArgs& a, const int* ag_r, cons
     }
   }
   const int len = rk.len;
-  for (int p0 = 0; p0 < len; p0 += 16) {
+  const int start = (m == 0) ? at : 0;
+  for (int p0 = start & ~15; p0 < len; p0 += 16) {
     const int c = p0 >> 4;
     uint4 cur = rk.ck[0];
     bool have = false;
@@ -282,8 +297,8 @@ __device__ __forceinline__ int propose(const PhaseArgs& a, const int* ag_r, cons
     if (!have)
       cur = reinterpret_cast<const uint4*>(a.pref + static_cast<size_t>(t) * pref_stride(a.E))[c];
     const uint32_t w4[4] = {cur.x, cur.y, cur.z, cur.w};
-    // all sixteen tests at once (entries past len are masked off afterwards; the index is
-    // clamped so that their bytes stay inside the excluded set's words)
+    // all sixteen tests at once (entries outside [start, len) are masked off afterwards; the
+    // index is clamped so that their bytes stay inside the excluded set's words)
     uint32_t avail = 0;
 #pragma unroll
     for (int b = 0; b < 16; ++b) {
@@ -294,19 +309,22 @@ __device__ __forceinline__ int propose(const PhaseArgs& a, const int* ag_r, cons
       avail |= bit << b;
     }
     if (len - p0 < 16) avail &= (1u << (len - p0)) - 1u;
+    if (start > p0) avail &= ~0u << (start - p0);
     const int na = __popc(avail);
     if (m < na) {
       for (int r = 0; r < m; ++r) avail &= avail - 1u;
       const int b = __ffs(avail) - 1;
       const uint32_t w = (b < 4) ? cur.x : (b < 8) ? cur.y : (b < 12) ? cur.z : cur.w;
+      at = p0 + b;
       return (w >> (8 * (b & 3))) & 0xff;
     }
     m -= na;
   }
+  at = len;
   return -1;
 }
 
-// The ranking of the token of pending route i into this SM's L1, ahead of a proposal.
+// The ranking of a pending route's token into this SM's L1, ahead of a proposal.
 __device__ __forceinline__ void prefetch_ranking(const PhaseArgs& a, int t) {
   const uint8_t* row = a.pref + static_cast<size_t>(t) * pref_stride(a.E);
   for (int off = 0; off < pref_stride(a.E); off += 128)
@@ -338,10 +356,12 @@ __global__ void __launch_bounds__(kPhThreads, 1) reroute_phase_kernel(PhaseArgs 
   const int E = a.E, k = a.k, C = a.C;
   const int total = a.T * k;  // <= INT_MAX / 2 (validated on the host)
   // pending routes in arrival order: token << 5 | slot, proposed / final expert (-1: none),
-  // and a flag set when an earlier route of the same token proposed again
+  // a flag set when an earlier route of the same token proposed again, and the position in
+  // the token's ranking of the last proposal
   int* ag_r = SMEM ? s_dyn : a.g_r;
   int* ag_c = SMEM ? s_dyn + total : a.g_c;
   uint8_t* dirty = SMEM ? reinterpret_cast<uint8_t*>(s_dyn + 2 * total) : a.g_dirty;
+  uint8_t* at = SMEM ? reinterpret_cast<uint8_t*>(s_dyn + 2 * total) + total : a.g_at;
   pdl_wait();
 
   for (int x = tid; x < kPhWarps * 257; x += kPhThreads) (&s_wc[0][0])[x] = 0;
@@ -387,7 +407,8 @@ __global__ void __launch_bounds__(kPhThreads, 1) reroute_phase_kernel(PhaseArgs 
       for (int u = 0; u < 16; ++u) {
         if ((bits >> u) & 1u) {
           ag_r[out] = (t << 5) | j;
-          ag_c[out] = v[u];
+          ag_c[out] = prop_expert(v[u]);
+          at[out] = static_cast<uint8_t>(prop_at(v[u]));
           dirty[out] = 0;
           ++out;
         }
@@ -436,7 +457,11 @@ __global__ void __launch_bounds__(kPhThreads, 1) reroute_phase_kernel(PhaseArgs 
           again = dirty[q] != 0 || (cq >= 0 && ((full[cq >> 5] >> (cq & 31)) & 1u));
         }
       }
-      if (again) c = propose<NW>(a, ag_r, ag_c, i, pos, full, s_ex + tid);
+      int at_i = 0;
+      if (again) {
+        at_i = at[i];
+        c = propose<NW>(a, ag_r, ag_c, i, pos, full, s_ex + tid, at_i);
+      }
       // scan in arrival order; place every route before the first one whose expert has no
       // slot left for it.  A route's rank among the block's proposals to its expert is its
       // rank in its warp plus the earlier warps' counts.
@@ -448,6 +473,7 @@ __global__ void __launch_bounds__(kPhThreads, 1) reroute_phase_kernel(PhaseArgs 
       __syncthreads();
       if (again) {
         ag_c[i] = c;
+        at[i] = static_cast<uint8_t>(at_i);
         dirty[i] = 0;
         const int t = tr >> 5;
         for (int q = i + 1; q < n && (ag_r[q] >> 5) == t; ++q)
@@ -502,7 +528,7 @@ __global__ void __launch_bounds__(kPhThreads, 1) reroute_phase_kernel(PhaseArgs 
   pdl_trigger();
 }
 
-constexpr int kRouteSmemBytes = 2 * sizeof(int) + 1;  // ag_r, ag_c, dirty
+constexpr int kRouteSmemBytes = 2 * sizeof(int) + 2;  // ag_r, ag_c, dirty, at
 
 template <int NW>
 cudaError_t launch_placement(const FirstArgs& fa, const PhaseArgs& pa, cudaStream_t s) {
@@ -592,7 +618,9 @@ cudaError_t launch_reroute(const moe_config& c, const void* x, const int32_t* id
                      pref_len, c.T, c.k,       c.E,     c.capacity};
   const PhaseArgs pa{zkeys, prop, pref, pref_len, row_token, route_row, offsets, list,
                      prop + routes, prop + 2 * routes,
-                     reinterpret_cast<uint8_t*>(prop + 3 * routes), c.T, c.k, c.E, c.capacity,
+                     reinterpret_cast<uint8_t*>(prop + 3 * routes),
+                     reinterpret_cast<uint8_t*>(prop + 3 * routes) + routes, c.T, c.k, c.E,
+                     c.capacity,
                      routes <= static_cast<size_t>(kSmemRoutes) ? 1 : 0};
   cudaError_t e = c.E <= 32   ? launch_placement<1>(fa, pa, s)
                   : c.E <= 64  ? launch_placement<2>(fa, pa, s)
