@@ -112,6 +112,37 @@ __device__ __forceinline__ void set_bit(uint32_t (&w)[NW], int e) {
     if (q == (e >> 5)) w[q] |= 1u << (e & 31);
 }
 
+// Ascending bitonic sort of 32 NW keys held by a warp, key q of lane l at position 32 q + l.
+template <int NW>
+__device__ __forceinline__ void warp_bitonic_sort(uint64_t (&v)[NW], int lane) {
+  constexpr int N = 32 * NW;
+#pragma unroll
+  for (int size = 2; size <= N; size <<= 1) {
+#pragma unroll
+    for (int j = size >> 1; j > 0; j >>= 1) {
+      if (j >= 32) {  // partner in another register of the same lane
+#pragma unroll
+        for (int q = 0; q < NW; ++q) {
+          const int p = q ^ (j >> 5);
+          if (p > q) {
+            const bool asc = ((32 * q + lane) & size) == 0;
+            const uint64_t x = v[q], y = v[p];
+            if ((x > y) == asc) { v[q] = y; v[p] = x; }
+          }
+        }
+      } else {  // partner in another lane
+#pragma unroll
+        for (int q = 0; q < NW; ++q) {
+          const uint64_t o = __shfl_xor_sync(0xffffffffu, v[q], j);
+          const bool asc = ((32 * q + lane) & size) == 0;
+          const bool take_min = ((lane & j) == 0) == asc;
+          v[q] = take_min ? (o < v[q] ? o : v[q]) : (o > v[q] ? o : v[q]);
+        }
+      }
+    }
+  }
+}
+
 struct FirstArgs {
   const int32_t* ids;      // [T, k]
   const float* zkeys;      // [T, E]
@@ -124,14 +155,13 @@ struct FirstArgs {
 };
 
 // One warp per token with an overflowed route.  It ranks the experts the token does not
-// hold (descending key, equal keys to the lower index; NaN keys rank as -inf), stores that
-// order, and makes the first proposals: with nothing placed yet, the token's overflowed
-// routes take, in slot order, the first, second, ... experts of the order that are not full
-// after the arrival-order pass.
+// hold (descending key, equal keys to the lower index; NaN keys rank as -inf) with a warp
+// bitonic sort, stores that order, and makes the first proposals: with nothing placed yet,
+// the token's overflowed routes take, in slot order, the first, second, ... experts of the
+// order that are not full after the arrival-order pass.
 template <int NW>
 __global__ void __launch_bounds__(kFirstWarps * 32) reroute_first_kernel(FirstArgs a) {
   __shared__ uint32_t s_full[8];
-  __shared__ float s_z[kFirstWarps][256];
   __shared__ uint32_t s_list[kFirstWarps][64];  // 256 expert bytes per warp
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int k = a.k, E = a.E, Ep = pref_stride(E);
@@ -166,30 +196,26 @@ __global__ void __launch_bounds__(kFirstWarps * 32) reroute_first_kernel(FirstAr
       held[w] = __reduce_or_sync(0xffffffffu, mine ? 1u << (id & 31) : 0u);
       nheld += __popc(held[w]);
     }
+    // sort keys: the key's order flipped (larger keys first; -0 as +0, NaN as -inf) above the
+    // expert index (equal keys: lower index first); held experts and e >= E sort last
     const float* zrow = a.zkeys + static_cast<size_t>(t) * E;
-    for (int e = lane; e < E; e += 32) {
-      const float v = zrow[e];
-      s_z[warp][e] = (v != v) ? -INFINITY : v;
-    }
-    __syncwarp();
+    uint64_t key[NW];
 #pragma unroll
     for (int q = 0; q < NW; ++q) {
       const int e = lane + 32 * q;
-      if (e >= E || ((held[q] >> lane) & 1u)) continue;
-      const float v = s_z[warp][e];
-      int rank = 0;
-#pragma unroll
-      for (int w = 0; w < NW; ++w) {
-#pragma unroll 8
-        for (int b = 0; b < 32; ++b) {
-          const int e2 = 32 * w + b;
-          if (e2 >= E || ((held[w] >> b) & 1u)) continue;
-          const float u = s_z[warp][e2];
-          rank += (u > v || (u == v && e2 < e)) ? 1 : 0;
-        }
+      key[q] = ~0ull;
+      if (e < E && !((held[q] >> lane) & 1u)) {
+        float v = zrow[e];
+        v = (v != v) ? -INFINITY : (v == 0.f ? 0.f : v);
+        const uint32_t u = __float_as_uint(v);
+        const uint32_t ordered = (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // ascending in v
+        key[q] = (static_cast<uint64_t>(~ordered) << 32) | static_cast<uint32_t>(e);
       }
-      lst[rank] = static_cast<uint8_t>(e);
     }
+    warp_bitonic_sort<NW>(key, lane);
+#pragma unroll
+    for (int q = 0; q < NW; ++q)  // position 32 q + lane of the ranking
+      lst[32 * q + lane] = static_cast<uint8_t>(key[q] & 0xffu);
     __syncwarp();
     const int len = E - nheld;
     uint32_t* dst = reinterpret_cast<uint32_t*>(a.pref + static_cast<size_t>(t) * Ep);
