@@ -381,6 +381,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------------
 constexpr int kCluster = 8;
 constexpr int kMaxSmemPerCta = 227 * 1024;
+constexpr int kSmemPerSm = 228 * 1024;      // shared memory of one SM
+constexpr int kSmemReservedPerCta = 1024;   // taken by the system from each resident CTA
 constexpr int kTokPerCta = kTokens / kCluster;  // 16
 constexpr int kLanesPerTok = 128 / kTokPerCta;  // 8
 
@@ -722,6 +724,11 @@ cudaError_t launch_router_sm100(const moe_config& c, const void* x, const void* 
     int cstages = (k_blocks + kCluster - 1) / kCluster;
     if (cstages > stages) cstages = stages;
     if (cstages > (kMaxSmemPerCta - fixed) / stage_bytes) cstages = (kMaxSmemPerCta - fixed) / stage_bytes;
+    // Two CTAs per SM where that still leaves a two-stage ring: a CTA spends most of its
+    // life in the cluster reduction and the top-k epilogue, which then overlap the other
+    // CTA's TMA stream (the whole grid rarely fits in one wave of one CTA per SM).
+    const int two_per_sm = (kSmemPerSm / 2 - kSmemReservedPerCta - fixed) / stage_bytes;
+    if (two_per_sm >= 2 && cstages > two_per_sm) cstages = two_per_sm;
     RouteParams pc = p;
     pc.stages = cstages;
     const int csmem = fixed + cstages * stage_bytes;
