@@ -724,11 +724,16 @@ cudaError_t launch_router_sm100(const moe_config& c, const void* x, const void* 
     int cstages = (k_blocks + kCluster - 1) / kCluster;
     if (cstages > stages) cstages = stages;
     if (cstages > (kMaxSmemPerCta - fixed) / stage_bytes) cstages = (kMaxSmemPerCta - fixed) / stage_bytes;
-    // Two CTAs per SM where that still leaves a two-stage ring: a CTA spends most of its
-    // life in the cluster reduction and the top-k epilogue, which then overlap the other
-    // CTA's TMA stream (the whole grid rarely fits in one wave of one CTA per SM).
-    const int two_per_sm = (kSmemPerSm / 2 - kSmemReservedPerCta - fixed) / stage_bytes;
-    if (two_per_sm >= 2 && cstages > two_per_sm) cstages = two_per_sm;
+    // As many CTAs per SM (up to 4) as still leave a two-stage ring: a CTA spends most of
+    // its life in the cluster reduction and the top-k epilogue, which then overlap the
+    // other CTAs' TMA streams (the grid rarely fits in one wave of one CTA per SM).
+    for (int per_sm = 4; per_sm >= 2; --per_sm) {
+      const int fit = (kSmemPerSm / per_sm - kSmemReservedPerCta - fixed) / stage_bytes;
+      if (fit >= 2) {
+        if (cstages > fit) cstages = fit;
+        break;
+      }
+    }
     RouteParams pc = p;
     pc.stages = cstages;
     const int csmem = fixed + cstages * stage_bytes;
