@@ -16,10 +16,10 @@ namespace moe {
 // Called by every thread of each CTA that wrote one tile's row of p.tile_hist, after the
 // writes.  `scratch` is shared memory of at least kPrepScratchInts ints that the CTA no
 // longer needs (the function declares no shared memory of its own, so a kernel that opts
-// into the whole dynamic shared-memory budget can still call it).  The CTA that arrives last replaces the histogram by per-tile exclusive prefixes
-// (tile_hist[i][e] = routes to e in tiles < i), writes demand, the segment table and the
-// filled-slot counts, and resets the ticket.  Returns after that CTA's work (others return
-// at once).
+// into the whole dynamic shared-memory budget can still call it).  The CTA that arrives
+// last replaces the histogram by per-tile exclusive prefixes (tile_hist[i][e] = routes to e
+// in tiles < i), writes demand, the segment table and the filled-slot counts, and resets the
+// ticket.  Returns after that CTA's work (others return at once).
 constexpr int kPrepScratchInts = 3 * 257 + 1;
 
 __device__ __forceinline__ void dispatch_prep_arrive(const DispatchPrep& p, int* scratch) {
@@ -43,12 +43,24 @@ __device__ __forceinline__ void dispatch_prep_arrive(const DispatchPrep& p, int*
   const int parts = nth / E >= 1 ? nth / E : 1;
   const int chunk = (nt + parts - 1) / parts;
   // 1. each pair sums its range of tiles (loads bypass L1: the rows were written by other
-  //    SMs during this kernel)
+  //    SMs during this kernel); a thread with a single pair of up to kKeep tiles keeps the
+  //    counts for step 3 instead of loading them again
+  constexpr int kKeep = 8;
+  const bool keep = parts * E <= nth && chunk <= kKeep;
+  int counts[kKeep];
   for (int w = tid; w < parts * E; w += nth) {
     const int e = w % E, part = w / E;
     const int i0 = part * chunk, i1 = min(nt, i0 + chunk);
     int sum = 0;
-    for (int i = i0; i < i1; ++i) sum += __ldcg(p.tile_hist + static_cast<size_t>(i) * E + e);
+    if (keep) {
+#pragma unroll
+      for (int q = 0; q < kKeep; ++q)
+        counts[q] = (i0 + q < i1) ? __ldcg(p.tile_hist + static_cast<size_t>(i0 + q) * E + e) : 0;
+#pragma unroll
+      for (int q = 0; q < kKeep; ++q) sum += counts[q];
+    } else {
+      for (int i = i0; i < i1; ++i) sum += __ldcg(p.tile_hist + static_cast<size_t>(i) * E + e);
+    }
     s_part[part * E + e] = sum;
   }
   __syncthreads();
@@ -68,11 +80,20 @@ __device__ __forceinline__ void dispatch_prep_arrive(const DispatchPrep& p, int*
     const int e = w % E, part = w / E;
     const int i0 = part * chunk, i1 = min(nt, i0 + chunk);
     int pre = s_part[part * E + e];
-    for (int i = i0; i < i1; ++i) {
-      int* q = p.tile_hist + static_cast<size_t>(i) * E + e;
-      const int h = __ldcg(q);
-      *q = pre;
-      pre += h;
+    if (keep) {
+#pragma unroll
+      for (int q = 0; q < kKeep; ++q)
+        if (i0 + q < i1) {
+          p.tile_hist[static_cast<size_t>(i0 + q) * E + e] = pre;
+          pre += counts[q];
+        }
+    } else {
+      for (int i = i0; i < i1; ++i) {
+        int* q = p.tile_hist + static_cast<size_t>(i) * E + e;
+        const int h = __ldcg(q);
+        *q = pre;
+        pre += h;
+      }
     }
   }
   // 4. kept counts -> segment starts (warp 0); the padded buffer gives expert e rows e*C ..
