@@ -370,7 +370,9 @@ def measure_workload(a, wl, dev, world, rank, e2e=False, cpu=False):
         raise RuntimeError(f"{wl.name}: device status {st} after warm-up")
 
     nprof = max(1, min(a.profiled_steps, a.steps))
-    evs = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
+    # one interval per step; the reroute policy's kernels get their own (seven events)
+    knames = (KERNELS[:2] + ["reroute"] + KERNELS[2:]) if wl.overflow == "reroute" else KERNELS
+    evs = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(knames) + 1)]
             for _ in range(L)] for _ in range(nprof)]
     for s_ in evs:  # create the handles before capture / timing
         for l_ in s_:
@@ -447,15 +449,15 @@ def measure_workload(a, wl, dev, world, rank, e2e=False, cpu=False):
             flush.zero_()
         profiled_step(i)
     torch.cuda.synchronize(dev)
-    per = {k: [] for k in KERNELS}
+    per = {k: [] for k in knames}
     for s in range(nprof):
         for l in range(L):
             e = evs[s][l]
-            for i, kname in enumerate(KERNELS):
+            for i, kname in enumerate(knames):
                 per[kname].append(e[i].elapsed_time(e[i + 1]))
     avg_ms = {k: statistics.mean(v) for k, v in per.items()}
     tot_ms = {k: sum(v) for k, v in per.items()}
-    dom = max(tot_ms, key=tot_ms.get)
+    dom = max(KERNELS, key=tot_ms.get)  # the kernels with an algorithmic-bytes model
 
     dem = demand.cpu()
     offs = offsets.cpu()
@@ -508,7 +510,11 @@ def measure_workload(a, wl, dev, world, rank, e2e=False, cpu=False):
     breakdown = {k: {"avg_us": round(avg_ms[k] * 1e3, 2), "share": round(tot_ms[k] / sum(tot_ms.values()), 4),
                      "frac": round(roof(k)["frac"], 4), "frac_of_spec": round(roof(k)["frac_of_spec"], 4),
                      "bound": roof(k)["bound"]} for k in KERNELS}
-    launches = L * ((7 if wl.overflow == "reroute" else 5) + int(a.stats)
+    if "reroute" in per:  # the placement is a latency chain: time and share only
+        breakdown["reroute"] = {"avg_us": round(avg_ms["reroute"] * 1e3, 2),
+                                "share": round(tot_ms["reroute"] / sum(tot_ms.values()), 4),
+                                "bound": "latency"}
+    launches = L * ((8 if wl.overflow == "reroute" else 5) + int(a.stats)
                     - (1 if "combine" in fuse else 0))
 
     out = {"workload": wl.name, "ms_per_step": ms_per_step,

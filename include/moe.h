@@ -235,8 +235,11 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
 
 /* moe_forward that also records caller-created CUDA events (cudaEvent_t handles, e.g.
  * created with timing enabled) on `stream` around its kernels, for live per-kernel timing:
- * events[0] before the first kernel, events[i] after kernel i, i = 1..5 in the order
- * route, pack, gate/up GEMM, down GEMM, combine.  n_events must be 6.                   */
+ * events[0] before the first kernel, events[i] after step i, i = 1..5 in the order
+ * route, pack (with the reroute policy's kernels), gate/up GEMM, down GEMM, combine, for
+ * n_events = 6; with n_events = 7 the reroute gets its own step after the pack (route,
+ * pack, reroute, gate/up, down, combine; an empty interval without the reroute policy).
+ * Any other n_events, or a NULL handle, is MOE_ERR_INVALID.                             */
 moe_status moe_forward_profiled(const moe_config* cfg, const void* x, const void* w_router,
                                 const float* logit_bias, const void* w_gate, const void* w_up,
                                 const void* w_down, const void* shared_gate,

@@ -147,7 +147,8 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
                         const float* logit_bias, const void* w_gate, const void* w_up,
                         const void* w_down, const void* shared_gate, const void* shared_up,
                         const void* shared_down, void* y, int32_t* ids_out, float* gates_out,
-                        int32_t* demand_out, int32_t* offsets_out, void* const* ev, void* ws,
+                        int32_t* demand_out, int32_t* offsets_out, void* const* ev, int n_ev,
+                        void* ws,
                         cudaStream_t stream) {
   MOE_TRY(validate(cfg));
   MOE_TRY(check_ws(ws));
@@ -173,6 +174,8 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
   // table, so the pack reads finished positions.
   const DispatchPrep prep = make_dispatch_prep(
       c, hist, offsets, demand, reinterpret_cast<unsigned int*>(at(ws, kWsPrepCounterOffset)));
+  // events: 0 start, then after route, pack, [reroute, with 7 events], gate/up, down, combine
+  const int rr_ev = (n_ev == 7) ? 1 : 0;
   MOE_TRY(record(ev, 0, stream));
   MOE_TRY(cuda_status(
       launch_router(c, x, w_router, logit_bias, ids, gates, hist, extra, prep, status, stream)));
@@ -187,21 +190,22 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
   MOE_TRY(cuda_status(launch_dispatch_pack(c, x, ids, hist, offsets, x_packed, row_token,
                                            route_row, status, stream,
                                            c.fuse != 0 ? &pf : nullptr)));
+  if (rr_ev) MOE_TRY(record(ev, 2, stream));
   if (reroute(c))
     MOE_TRY(cuda_status(launch_reroute(c, x, ids, extra.zkeys, gates, x_packed, row_token,
                                        route_row, offsets,
                                        reinterpret_cast<int32_t*>(at(ws, L.rlist)), status,
                                        stream)));
-  MOE_TRY(record(ev, 2, stream));
+  MOE_TRY(record(ev, 2 + rr_ev, stream));
   const FusedCombine fc{route_row, gates, row_token, need, counters, resid, y, c.k, c.has_shared};
   FfnArgs f{x, x_packed, offsets, w_gate, w_up, w_down, shared_gate, shared_up, shared_down,
             h, y_packed, L.rmax, status, padded(c) ? offsets + c.E + 2 : nullptr,
             fuse_gather ? row_token : nullptr, fuse_combine ? &fc : nullptr};
-  MOE_TRY(ffn(c, f, stream, ev ? static_cast<cudaEvent_t>(ev[3]) : nullptr));
-  MOE_TRY(record(ev, 4, stream));
+  MOE_TRY(ffn(c, f, stream, ev ? static_cast<cudaEvent_t>(ev[3 + rr_ev]) : nullptr));
+  MOE_TRY(record(ev, 4 + rr_ev, stream));
   if (!fuse_combine)
     MOE_TRY(cuda_status(launch_combine(c, y_packed, route_row, gates, offsets, x, y, stream)));
-  return record(ev, 5, stream);
+  return record(ev, 5 + rr_ev, stream);
 }
 
 }  // namespace
@@ -321,8 +325,8 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
                        int32_t* demand_out, int32_t* offsets_out, void* ws,
                        moe_stream_t stream) {
   return forward_impl(cfg, x, w_router, logit_bias, w_gate, w_up, w_down, shared_gate, shared_up,
-                      shared_down, y, ids_out, gates_out, demand_out, offsets_out, nullptr, ws,
-                      stream);
+                      shared_down, y, ids_out, gates_out, demand_out, offsets_out, nullptr, 0,
+                      ws, stream);
 }
 
 moe_status moe_forward_profiled(const moe_config* cfg, const void* x, const void* w_router,
@@ -332,12 +336,12 @@ moe_status moe_forward_profiled(const moe_config* cfg, const void* x, const void
                                 int32_t* ids_out, float* gates_out, int32_t* demand_out,
                                 int32_t* offsets_out, void* const* events, int32_t n_events,
                                 void* ws, moe_stream_t stream) {
-  if (events == nullptr || n_events != 6) return MOE_ERR_INVALID;
-  for (int i = 0; i < 6; ++i)
+  if (events == nullptr || (n_events != 6 && n_events != 7)) return MOE_ERR_INVALID;
+  for (int i = 0; i < n_events; ++i)
     if (events[i] == nullptr) return MOE_ERR_INVALID;
   return forward_impl(cfg, x, w_router, logit_bias, w_gate, w_up, w_down, shared_gate, shared_up,
-                      shared_down, y, ids_out, gates_out, demand_out, offsets_out, events, ws,
-                      stream);
+                      shared_down, y, ids_out, gates_out, demand_out, offsets_out, events,
+                      n_events, ws, stream);
 }
 
 moe_status moe_routing_stats(const moe_config* cfg, const int32_t* demand,

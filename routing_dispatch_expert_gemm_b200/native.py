@@ -217,11 +217,12 @@ def moe_forward(cfg, x, w_router, logit_bias, w_gate, w_up, w_down, shared_gate,
 def moe_forward_profiled(cfg, x, w_router, logit_bias, w_gate, w_up, w_down, shared_gate,
                          shared_up, shared_down, y, ids_out, gates_out, demand_out, offsets_out,
                          events, ws, stream=None):
-    """``events``: six torch.cuda.Event objects (or raw cudaEvent_t handles as ints)."""
+    """``events``: six (or seven) torch.cuda.Event objects, or raw cudaEvent_t handles as
+    ints; see moe_forward_profiled in include/moe.h."""
     for e in events:  # torch creates an event's handle at its first record
         if not isinstance(e, int) and e.cuda_event == 0:
             e.record()
-    handles = (_P * 6)(*[e if isinstance(e, int) else e.cuda_event for e in events])
+    handles = (_P * len(events))(*[e if isinstance(e, int) else e.cuda_event for e in events])
     _check(lib().moe_forward_profiled(ctypes.byref(cfg), _ptr(x), _ptr(w_router),
                                       _ptr(logit_bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
                                       _ptr(shared_gate), _ptr(shared_up), _ptr(shared_down),

@@ -106,6 +106,16 @@ def test_errors_return_before_any_launch(native):
                               None, fake, fake, 4096, None) == 1
     assert lib.moe_forward(ctypes.byref(cfg), fake, fake, None, fake, fake, fake, None, None,
                            None, None, None, None, None, None, 4096, None) == 1
+    # moe_forward_profiled takes 6 or 7 events, none of them NULL
+    evs = (ctypes.c_void_p * 8)(*([fake] * 8))
+    prof = lambda events, n: lib.moe_forward_profiled(
+        ctypes.byref(cfg), fake, fake, None, fake, fake, fake, None, None, None, fake, None,
+        None, None, None, events, n, 4096, None)
+    for n in (0, 5, 8):
+        assert prof(evs, n) == 1
+    assert prof(None, 6) == 1
+    holed = (ctypes.c_void_p * 7)(*([fake] * 6 + [None]))
+    assert prof(holed, 7) == 1
     assert lib.moe_debug_bounded_wait(4096, 10, None) == 1
     assert native.moe_status_string(6).startswith("a bounded")
 

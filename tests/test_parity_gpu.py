@@ -433,3 +433,23 @@ def test_forward_profiled_matches_forward_and_times_kernels():
     assert torch.equal(y2, ref["y"])
     assert all(evs[i].elapsed_time(evs[i + 1]) > 0 for i in range(5))
     assert N.moe_get_device_status(ws) == 0
+
+
+def test_forward_profiled_seven_events_times_the_reroute():
+    """With seven events the reroute policy's kernels get their own interval; the bits are
+    those of moe_forward."""
+    wl = W["switch_phi125_reroute"].with_(T=512)
+    x, (p,) = I.make_inputs(wl, seed=6, device="cuda", layers=1)
+    cfg = config_for(wl)
+    ref = forward_gpu(cfg, x, p)
+    ws = N.workspace(cfg)
+    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(7)]
+    y = torch.empty_like(x)
+    N.moe_forward_profiled(cfg, x, p["w_router"], p["logit_bias"], p["w_gate"], p["w_up"],
+                           p["w_down"], p["shared_gate"], p["shared_up"], p["shared_down"], y,
+                           None, None, None, None, evs, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y, ref["y"])
+    times = [evs[i].elapsed_time(evs[i + 1]) for i in range(6)]
+    assert all(t > 0 for t in times), times
+    assert N.moe_get_device_status(ws) == 0
