@@ -104,14 +104,6 @@ __host__ __device__ constexpr int prop_at(int v) { return v >> 16; }
 
 __host__ __device__ constexpr int pref_stride(int E) { return (E + 15) & ~15; }
 
-// Expert bit sets over NW words (bits at e >= E set where the set means "excluded").
-template <int NW>
-__device__ __forceinline__ void set_bit(uint32_t (&w)[NW], int e) {
-#pragma unroll
-  for (int q = 0; q < NW; ++q)
-    if (q == (e >> 5)) w[q] |= 1u << (e & 31);
-}
-
 // Ascending bitonic sort of 32 NW keys held by a warp, key q of lane l at position 32 q + l.
 template <int NW>
 __device__ __forceinline__ void warp_bitonic_sort(uint64_t (&v)[NW], int lane) {

@@ -91,6 +91,9 @@ REROUTE_CASES = {
     "C0": (64, 128, 4, 2, (0, 1), None, "topk_softmax", "bf16"),
     # 16384 routes, many overflowing: a long cascade of placement phases
     "E16_k4_many_phases": (4096, 128, 16, 4, (1, 1), [3, 2, 1] + [0] * 13, "softmax_topk_renorm", "bf16"),
+    # 24000 routes: above what the placement keeps in shared memory, so its pending-route
+    # arrays live in global memory
+    "E16_k4_global_arrays": (6000, 128, 16, 4, (1, 1), [2, 2, 1] + [0] * 13, "topk_softmax", "bf16"),
 }
 
 
