@@ -22,7 +22,6 @@ namespace {
 constexpr int kThreads = 256;  // copy kernel
 constexpr int kWarps = kThreads / 32;
 
-
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int s = 16; s >= 1; s >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, s));
