@@ -43,6 +43,9 @@ SMALL = {
     "shared64_narrow_phi1": W["shared64_T256_phi1"].with_(T=300, d=512, d_ff=1024),
     "shared64_narrow_dropless": W["shared64_T256_dropless"].with_(T=300, d=512, d_ff=1024),
     "shared64_narrow_phi2_T1": W["shared64_T1_phi2"].with_(d=512, d_ff=1024),
+    # about 128 rows per routed expert: segments just above one 128-row tile (two tiles, the
+    # second nearly empty) next to smaller and larger ones, and a 1024-row shared segment
+    "shared16_narrow": W["shared16_T1024_F8192"].with_(d=512, d_ff=1024),
 }
 
 
@@ -173,7 +176,7 @@ def test_layer_parity_on_oracle_routing(name):
 @pytest.mark.parametrize("tiles", ["rows", "columns", "pairs"])
 @pytest.mark.parametrize("name", ["granite_layer", "switch_phi125", "switch_phi050", "mixtral_T300",
                                   "mixtral_decode", "shared64_narrow_phi1",
-                                  "shared64_narrow_phi2_T1"])
+                                  "shared64_narrow_phi2_T1", "shared16_narrow"])
 def test_both_tile_shapes_on_oracle_routing(name, tiles):
     """The row-tile, column-tile and SM-pair FFN kernels, forced on the same inputs and
     routing, each against the oracle (segments of 1 to a few hundred rows, ragged tails, the
