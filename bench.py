@@ -49,9 +49,9 @@ KERNELS = ["route", "pack", "gemm_gate_up", "gemm_down", "combine"]
 KERNEL_SOURCES = {"route": ["route.cu", "route_sm100.cu", "dispatch_prep.cuh", "common.cuh"],
                   "pack": ["dispatch.cu", "dispatch_prep.cuh", "reroute.cu", "common.cuh"],
                   "gemm_gate_up": ["gemm_sm100.cu", "gemm_cols_sm100.cu", "gemm_pair_sm100.cu",
-                                   "gemm_common.cuh", "common.cuh"],
+                                   "gemm_rowpair_sm100.cu", "gemm_common.cuh", "common.cuh"],
                   "gemm_down": ["gemm_sm100.cu", "gemm_cols_sm100.cu", "gemm_pair_sm100.cu",
-                                "gemm_common.cuh", "common.cuh"],
+                                "gemm_rowpair_sm100.cu", "gemm_common.cuh", "common.cuh"],
                   "combine": ["combine.cu", "common.cuh"]}
 
 

@@ -82,19 +82,27 @@ typedef enum {
                              * slot (MOE_LAYOUT_PADDED only; see moe_dispatch)              */
 } moe_overflow;
 
-/* Tile shape of the bf16 expert-FFN GEMMs (the fp32 configuration ignores it).  Both give
- * the same products; they differ in how ragged expert segments are padded.            */
+/* Tile shape of the bf16 expert-FFN GEMMs (the fp32 configuration ignores it).  All give
+ * the same products; they differ in how ragged expert segments are padded and in how many
+ * operand bytes each SM stages per k-block.                                               */
 typedef enum {
-  MOE_TILES_AUTO = 0,    /* row tiles (measured faster than column tiles on every workload
-                          * here), column tiles when a fused step is requested            */
+  MOE_TILES_AUTO = 0,    /* row tiles over SM pairs when the routed experts average at
+                          * least 512 rows each (C rows with the padded layout, else
+                          * min(C, T k / E)) and d % 256 == 0, d_ff % 128 == 0; else row
+                          * tiles; column tiles when a fused step is requested            */
   MOE_TILES_ROWS = 1,    /* 128 tokens x 256 output columns per tile: tokens on the MMA's M
                           * side; a segment is padded to a multiple of 128 rows           */
   MOE_TILES_COLUMNS = 2, /* 128 weight rows x up to 128 tokens per tile: weights on M,
                           * tokens on N; a segment is padded to a multiple of 16 rows     */
-  MOE_TILES_PAIRS = 3    /* column tiles over a pair of SMs (one M = 256 MMA, each SM
+  MOE_TILES_PAIRS = 3,   /* column tiles over a pair of SMs (one M = 256 MMA, each SM
                           * holding half of the token tile); a segment is padded to a
                           * multiple of 32 rows; needs d and d_ff multiples of 256, else
                           * row tiles run                                                  */
+  MOE_TILES_ROW_PAIRS = 4 /* row tiles over a pair of SMs: 256 tokens x 256 output columns
+                          * per pair tile (one M = 256 MMA; each SM holds 128 tokens and
+                          * half of the weight rows); a segment is padded to a multiple of
+                          * 256 rows; needs d % 256 == 0 and d_ff % 128 == 0, else row
+                          * tiles run                                                      */
 } moe_tiles;
 
 /* Steps of moe_forward fused into the expert GEMMs (bit flags; bf16, column tiles, drop
@@ -129,7 +137,8 @@ typedef struct {
   int32_t tiles;        /* moe_tiles (0 = automatic)                                     */
   int32_t fuse;         /* moe_fuse flags (0 = none); any flag selects column tiles and
                          * needs MOE_BF16 and MOE_OVERFLOW_DROP (else MOE_ERR_UNSUPPORTED);
-                         * MOE_TILES_ROWS with a flag is MOE_ERR_INVALID                  */
+                         * MOE_TILES_ROWS or MOE_TILES_ROW_PAIRS with a flag is
+                         * MOE_ERR_INVALID                                                */
 } moe_config;
 /* Supported shapes (else MOE_ERR_UNSUPPORTED): bf16 needs d % 128 == 0 and
  * d_ff % 128 == 0; fp32 needs d % 4 == 0 and d_ff % 4 == 0.                            */
@@ -150,8 +159,9 @@ int64_t moe_max_rows(const moe_config* cfg);
  * Returns 0 for an invalid config.                                                      */
 size_t moe_workspace_bytes(const moe_config* cfg);
 
-/* The FFN tile shape a config runs with: MOE_TILES_ROWS or MOE_TILES_COLUMNS (cfg->tiles,
- * or the automatic choice when it is MOE_TILES_AUTO); 0 for an invalid config.  Host-only. */
+/* The FFN tile shape a config runs with: one of MOE_TILES_ROWS .. MOE_TILES_ROW_PAIRS
+ * (cfg->tiles when its shape requirements hold, else row tiles; the automatic choice when
+ * it is MOE_TILES_AUTO); 0 for an invalid config.  Host-only.                            */
 int32_t moe_ffn_tile_shape(const moe_config* cfg);
 
 /* Zero the status word and scratch header of a workspace (async on `stream`).          */

@@ -21,7 +21,8 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_PATH = os.path.join(HERE, "libmoe.so")
 
 SOURCES = ["api.cu", "route.cu", "route_sm100.cu", "dispatch.cu", "reroute.cu", "gemm_simt.cu",
-           "gemm_sm100.cu", "gemm_cols_sm100.cu", "gemm_pair_sm100.cu", "combine.cu", "stats.cu",
+           "gemm_sm100.cu", "gemm_cols_sm100.cu", "gemm_pair_sm100.cu",
+           "gemm_rowpair_sm100.cu", "combine.cu", "stats.cu",
            "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",

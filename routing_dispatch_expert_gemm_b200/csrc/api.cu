@@ -27,9 +27,10 @@ moe_status validate_config(const moe_config* c) {
   if ((c->layout != MOE_LAYOUT_RAGGED && c->layout != MOE_LAYOUT_PADDED) ||
       (c->overflow != MOE_OVERFLOW_DROP && c->overflow != MOE_OVERFLOW_REROUTE))
     return MOE_ERR_INVALID;
-  if (c->tiles < MOE_TILES_AUTO || c->tiles > MOE_TILES_PAIRS) return MOE_ERR_INVALID;
+  if (c->tiles < MOE_TILES_AUTO || c->tiles > MOE_TILES_ROW_PAIRS) return MOE_ERR_INVALID;
   if (c->fuse < 0 || c->fuse > (MOE_FUSE_GATHER | MOE_FUSE_COMBINE)) return MOE_ERR_INVALID;
-  if (c->fuse != 0 && c->tiles == MOE_TILES_ROWS) return MOE_ERR_INVALID;
+  if (c->fuse != 0 && (c->tiles == MOE_TILES_ROWS || c->tiles == MOE_TILES_ROW_PAIRS))
+    return MOE_ERR_INVALID;
   if (c->fuse != 0 && (c->dtype != MOE_BF16 || c->overflow != MOE_OVERFLOW_DROP))
     return MOE_ERR_UNSUPPORTED;
   if (c->layout == MOE_LAYOUT_PADDED && c->capacity < 0) return MOE_ERR_INVALID;  // C sizes it

@@ -24,6 +24,8 @@
 // Every wait is bounded (mbar_wait_bounded): if one runs out, the CTA records
 // MOE_ERR_TIMEOUT, drains its own copies and MMAs, frees its tensor memory and returns.
 // No TMA multicast is used.
+#include <algorithm>
+
 #include "gemm_common.cuh"
 #include "internal.h"
 
@@ -357,16 +359,31 @@ int sm_count() {
   return v;
 }
 
-// Automatic tile shape: row tiles.  Column tiles cut the padding of small expert segments
-// (a 130-row segment costs 256 rows of row-tile MMA work but 144 token columns), but their
-// N <= 128 MMAs read about a third more shared memory per FLOP than the row tiles' N = 256
-// ones, and on B200 that costs more than the padding saves on every workload measured here
-// (the 64+1 layer at T = 4096, the Granite- and Mixtral-shaped layers, decode).  They stay
-// selectable, and they carry the fused gather and combine.
+// Automatic tile shape: row tiles, or row tiles over SM pairs when the routed experts'
+// segments are large.  Column tiles cut the padding of small expert segments (a 130-row
+// segment costs 256 rows of row-tile MMA work but 144 token columns), but their N <= 128
+// MMAs read about a third more shared memory per FLOP than the row tiles' N = 256 ones, and
+// on B200 that costs more than the padding saves on every workload measured here.  They
+// stay selectable, and they carry the fused gather and combine.  Row tiles over SM pairs
+// stage 32 KB per SM and k-block instead of 48 KB (six k-blocks in flight instead of four):
+// faster where segments fill several 256-row pair tiles (Mixtral-shaped prefill, ~2048 rows
+// per expert: 4.30 -> 4.13 ms; Switch-shaped layers, ~1024: 4-5%), slower where half of a
+// pair tile would be padding (the 64+1 layer at T = 4096, ~128 rows: +16%; decode: +13%;
+// the Granite-shaped layer, ~353 rows: +6%).
+bool row_pairs_fit(const moe_config& c) { return c.d % 256 == 0 && c.d_ff % 128 == 0; }
+
 int32_t ffn_tile_shape(const moe_config& c) {
   if (c.fuse != 0) return MOE_TILES_COLUMNS;  // the fused steps live in the column kernel
   if (c.tiles == MOE_TILES_COLUMNS) return MOE_TILES_COLUMNS;
   if (c.tiles == MOE_TILES_PAIRS && c.d % 256 == 0 && c.d_ff % 256 == 0) return MOE_TILES_PAIRS;
+  if (c.tiles == MOE_TILES_ROW_PAIRS && row_pairs_fit(c)) return MOE_TILES_ROW_PAIRS;
+  if (c.tiles == MOE_TILES_AUTO && row_pairs_fit(c)) {
+    // average rows of a routed expert's segment
+    int64_t rows = static_cast<int64_t>(c.T) * c.k / c.E;
+    if (c.capacity >= 0)
+      rows = (c.layout == MOE_LAYOUT_PADDED) ? c.capacity : std::min<int64_t>(rows, c.capacity);
+    if (rows >= 512) return MOE_TILES_ROW_PAIRS;
+  }
   return MOE_TILES_ROWS;
 }
 
@@ -375,6 +392,7 @@ cudaError_t launch_ffn_sm100(const moe_config& c, const FfnArgs& f, cudaStream_t
   const int32_t shape = ffn_tile_shape(c);
   if (shape == MOE_TILES_COLUMNS) return launch_ffn_cols_sm100(c, f, s, mid);
   if (shape == MOE_TILES_PAIRS) return launch_ffn_pair_sm100(c, f, s, mid);
+  if (shape == MOE_TILES_ROW_PAIRS) return launch_ffn_rowpair_sm100(c, f, s, mid);
   const int nseg = c.E + (c.has_shared ? 1 : 0);
   const long long rows_h = f.rmax + (c.has_shared ? c.T : 0);
   const long long mt_bound = (rows_h + BM - 1) / BM + nseg;

@@ -154,6 +154,9 @@ cudaError_t launch_ffn_cols_sm100(const moe_config& c, const FfnArgs& a, cudaStr
 // Column tiles over SM pairs (gemm_pair_sm100.cu); d and d_ff multiples of 256.
 cudaError_t launch_ffn_pair_sm100(const moe_config& c, const FfnArgs& a, cudaStream_t s,
                                   cudaEvent_t mid = nullptr);
+// Row tiles over SM pairs (gemm_rowpair_sm100.cu); d a multiple of 256, d_ff of 128.
+cudaError_t launch_ffn_rowpair_sm100(const moe_config& c, const FfnArgs& a, cudaStream_t s,
+                                     cudaEvent_t mid = nullptr);
 
 cudaError_t launch_debug_wait(int32_t* status, int64_t limit_ns, cudaStream_t s);
 

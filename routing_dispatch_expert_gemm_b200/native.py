@@ -21,7 +21,7 @@ DTYPES = {"f32": 0, "bf16": 1}
 GATE_MODES = {"softmax_topk": 0, "softmax_topk_renorm": 1, "topk_softmax": 2}
 LAYOUTS = {"ragged": 0, "padded": 1}
 OVERFLOWS = {"drop": 0, "reroute": 1}
-TILES = {"auto": 0, "rows": 1, "columns": 2, "pairs": 3}
+TILES = {"auto": 0, "rows": 1, "columns": 2, "pairs": 3, "row_pairs": 4}
 FUSE = {"none": 0, "gather": 1, "combine": 2, "gather+combine": 3}
 
 # Every symbol include/moe.h declares (checked by the CPU test suite).
@@ -163,11 +163,11 @@ def moe_max_rows(cfg: MoeConfig) -> int:
 
 
 def moe_ffn_tile_shape(cfg: MoeConfig) -> str:
-    """'rows' or 'columns': the FFN tile shape the config runs with."""
+    """'rows', 'columns', 'pairs' or 'row_pairs': the FFN tile shape the config runs with."""
     v = lib().moe_ffn_tile_shape(ctypes.byref(cfg))
     if v == 0:
         raise MoeError(1, "moe_ffn_tile_shape")
-    return {1: "rows", 2: "columns", 3: "pairs"}[v]
+    return {1: "rows", 2: "columns", 3: "pairs", 4: "row_pairs"}[v]
 
 
 def moe_workspace_bytes(cfg: MoeConfig) -> int:

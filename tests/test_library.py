@@ -206,11 +206,24 @@ def test_config_sweep_validation_and_sizes(native):
 
 
 def test_ffn_tile_shape_choice(native):
-    """Automatic tile shape: row tiles; column tiles when asked for or when a fused step is
-    requested; bad values and row tiles with fusion rejected."""
+    """Automatic tile shape: row tiles over SM pairs when the routed experts average at least
+    512 rows (Mixtral- and Switch-shaped layers), else row tiles (the 64+1 layer, decode, the
+    Granite-shaped layer); column tiles when asked for or when a fused step is requested;
+    bad values and row tiles with fusion rejected."""
     mk = native.make_config
     assert native.moe_ffn_tile_shape(mk(4096, 4096, 64, 2, 32768, has_shared=True)) == "rows"
     assert native.moe_ffn_tile_shape(mk(16, 4096, 8, 2, 14336)) == "rows"
+    assert native.moe_ffn_tile_shape(mk(1412, 1024, 32, 8, 512)) == "rows"
+    assert native.moe_ffn_tile_shape(mk(8192, 4096, 8, 2, 14336)) == "row_pairs"
+    assert native.moe_ffn_tile_shape(mk(4096, 768, 4, 1, 2432)) == "row_pairs"
+    assert native.moe_ffn_tile_shape(mk(4096, 768, 4, 1, 2432, capacity=512)) == "row_pairs"
+    assert native.moe_ffn_tile_shape(mk(4096, 768, 4, 1, 2432, capacity=511)) == "rows"
+    assert native.moe_ffn_tile_shape(mk(2048, 640, 4, 1, 2432)) == "rows"  # d % 256
+    assert native.moe_ffn_tile_shape(mk(8192, 4096, 8, 2, 14336, tiles="rows")) == "rows"
+    assert native.moe_ffn_tile_shape(mk(16, 4096, 8, 2, 14336, tiles="row_pairs")) == "row_pairs"
+    assert native.moe_ffn_tile_shape(mk(16, 640, 8, 2, 1024, tiles="row_pairs")) == "rows"
+    assert native.moe_workspace_bytes(mk(8192, 4096, 8, 2, 14336, tiles="row_pairs",
+                                         fuse="gather")) == 0
     assert native.moe_ffn_tile_shape(mk(8192, 4096, 8, 2, 14336, tiles="columns")) == "columns"
     assert native.moe_ffn_tile_shape(mk(16, 4096, 8, 2, 14336, tiles="rows")) == "rows"
     assert native.moe_ffn_tile_shape(mk(16, 4096, 8, 2, 14336, tiles="pairs")) == "pairs"
@@ -222,6 +235,6 @@ def test_ffn_tile_shape_choice(native):
     assert native.moe_workspace_bytes(mk(1412, 1024, 32, 8, 512, fuse="combine")) > \
         native.moe_workspace_bytes(mk(1412, 1024, 32, 8, 512))
     bad = mk(16, 4096, 8, 2, 14336)
-    bad.tiles = 4
+    bad.tiles = 5
     assert native.lib().moe_ffn_tile_shape(ctypes.byref(bad)) == 0
     assert native.moe_workspace_bytes(bad) == 0

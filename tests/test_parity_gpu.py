@@ -173,15 +173,15 @@ def test_layer_parity_on_oracle_routing(name):
     assert_close(out["y"], y_ref, wl.dtype, name)
 
 
-@pytest.mark.parametrize("tiles", ["rows", "columns", "pairs"])
+@pytest.mark.parametrize("tiles", ["rows", "columns", "pairs", "row_pairs"])
 @pytest.mark.parametrize("name", ["granite_layer", "switch_phi125", "switch_phi050", "mixtral_T300",
                                   "mixtral_decode", "shared64_narrow_phi1",
                                   "shared64_narrow_phi2_T1", "shared16_narrow"])
 def test_both_tile_shapes_on_oracle_routing(name, tiles):
-    """The row-tile, column-tile and SM-pair FFN kernels, forced on the same inputs and
-    routing, each against the oracle (segments of 1 to a few hundred rows, ragged tails, the
-    shared expert, capacity drops; the Switch-shaped layers' d = 768 runs row tiles when
-    pairs are asked for)."""
+    """The row-tile, column-tile, column-pair and row-pair FFN kernels, forced on the same
+    inputs and routing, each against the oracle (segments of 1 to a few thousand rows,
+    ragged tails, the shared expert, capacity drops; the Switch-shaped layers' d = 768 runs
+    row tiles when column pairs are asked for)."""
     wl, x, p, C, ids_ref, g32, out = _run_oracle_routing(SMALL[name], tiles=tiles)
     assert out["status"] == 0
     y_ref, _ = O.moe_layer(x, p, wl.k, wl.gate_mode, C, add_residual=wl.add_residual,
@@ -319,7 +319,8 @@ def _robust_tokens(info, ok, n_near, C):
 # ------------------------------------------------------------------------- full size
 
 @pytest.mark.parametrize("name,sample,tiles", [
-    ("mixtral_prefill", None, ("auto", "columns", "pairs")), ("mixtral_decode", None, ("auto", "pairs")),
+    ("mixtral_prefill", None, ("auto", "rows", "columns", "pairs")),
+    ("mixtral_decode", None, ("auto", "pairs", "row_pairs")),
     ("shared64_T16_dropless", None, ("auto", "fused")),
     ("shared64_T4096_dropless", 512, ("auto", "columns", "pairs", "fused")),
     ("shared64_T4096_phi1", 64, ("auto",)), ("switch_phi050", None, ("auto", "rows"))])
