@@ -514,7 +514,7 @@ def measure_workload(a, wl, dev, world, rank, e2e=False, cpu=False):
         breakdown["reroute"] = {"avg_us": round(avg_ms["reroute"] * 1e3, 2),
                                 "share": round(tot_ms["reroute"] / sum(tot_ms.values()), 4),
                                 "bound": "latency"}
-    launches = L * ((8 if wl.overflow == "reroute" else 5) + int(a.stats)
+    launches = L * ((6 if wl.overflow == "reroute" else 3) + N.moe_ffn_launches(cfg) + int(a.stats)
                     - (1 if "combine" in fuse else 0))
 
     out = {"workload": wl.name, "ms_per_step": ms_per_step,

@@ -89,7 +89,9 @@ typedef enum {
   MOE_TILES_AUTO = 0,    /* row tiles over SM pairs when the routed experts average at
                           * least 512 rows each (C rows with the padded layout, else
                           * min(C, T k / E)) and d % 256 == 0, d_ff % 128 == 0; else row
-                          * tiles; column tiles when a fused step is requested            */
+                          * tiles, with a shared expert of T >= 512 rows on row tiles over
+                          * SM pairs in launches of its own (moe_ffn_launches); column
+                          * tiles when a fused step is requested                           */
   MOE_TILES_ROWS = 1,    /* 128 tokens x 256 output columns per tile: tokens on the MMA's M
                           * side; a segment is padded to a multiple of 128 rows           */
   MOE_TILES_COLUMNS = 2, /* 128 weight rows x up to 128 tokens per tile: weights on M,
@@ -163,6 +165,12 @@ size_t moe_workspace_bytes(const moe_config* cfg);
  * (cfg->tiles when its shape requirements hold, else row tiles; the automatic choice when
  * it is MOE_TILES_AUTO); 0 for an invalid config.  Host-only.                            */
 int32_t moe_ffn_tile_shape(const moe_config* cfg);
+
+/* Kernel launches of the expert FFN (moe_expert_ffn, and that step of moe_forward) for the
+ * config: 2 (gate/up with SwiGLU, then down), or 4 when the automatic choice runs a shared
+ * expert of at least 512 rows (T >= 512) on row tiles over SM pairs, in launches of its own,
+ * while the routed segments take row tiles; 0 for an invalid config.  Host-only.          */
+int32_t moe_ffn_launches(const moe_config* cfg);
 
 /* Zero the status word and scratch header of a workspace (async on `stream`).          */
 moe_status moe_workspace_init(void* ws, moe_stream_t stream);

@@ -241,6 +241,11 @@ int32_t moe_ffn_tile_shape(const moe_config* cfg) {
   return ffn_tile_shape(*cfg);
 }
 
+int32_t moe_ffn_launches(const moe_config* cfg) {
+  if (validate(cfg) != MOE_OK) return 0;
+  return ffn_launches(*cfg);
+}
+
 int64_t moe_max_rows(const moe_config* cfg) {
   if (validate(cfg) != MOE_OK) return 0;
   return max_rows(*cfg);

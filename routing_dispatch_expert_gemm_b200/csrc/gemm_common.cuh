@@ -45,11 +45,14 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 // Segment table in shared memory, built by one warp: row starts s_row0[0..nseg], row
 // counts s_rows[0..nseg) (from `counts` for routed segments when given, else the gap to
 // the next start) and the exclusive prefix s_pre[0..nseg] of the tiles of each segment,
-// tiles = ceil(rows / rows_per_tile) * blocks_per_row_tile.
+// tiles = ceil(rows / rows_per_tile) * blocks_per_row_tile, or 0 for the segments a launch
+// leaves to another one (the routed segments s < E unless `routed`, the shared expert's
+// segment unless `shared`).
 __device__ __forceinline__ void build_segment_table(const int32_t* offsets, const int32_t* counts,
                                                     int nseg, int E, int rows_per_tile,
                                                     int blocks, int* s_pre, int* s_row0,
-                                                    int* s_rows) {
+                                                    int* s_rows, bool routed = true,
+                                                    bool shared = true) {
   const int lane = threadIdx.x & 31;
   for (int i = lane; i <= nseg; i += 32) s_row0[i] = __ldg(offsets + i);
   __syncwarp();
@@ -60,7 +63,8 @@ __device__ __forceinline__ void build_segment_table(const int32_t* offsets, cons
   for (int b = 0; b < nseg; b += 32) {
     const int s = b + lane;
     int t = 0;
-    if (s < nseg) t = ((s_rows[s] + rows_per_tile - 1) / rows_per_tile) * blocks;
+    if (s < nseg && (s < E ? routed : shared))
+      t = ((s_rows[s] + rows_per_tile - 1) / rows_per_tile) * blocks;
     int incl = t;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {

@@ -70,6 +70,7 @@ struct RowPairParams {
   int ldo;
   int32_t* status;
   int64_t limit_ns;
+  int routed, shared;     // which segments this launch runs (see build_segment_table)
 };
 
 template <int MODE>  // 0: SwiGLU gate|up; 1: down
@@ -121,7 +122,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_wait();  // offsets, A rows and the output buffer belong to earlier kernels
   if (warp == 0)
     gemm::build_segment_table(p.offsets, p.counts, p.nseg, p.E, 2 * BM, n_blocks, s_pre, s_row0,
-                              s_rows);
+                              s_rows, p.routed != 0, p.shared != 0);
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();  // both CTAs' barriers are initialised before any remote use
@@ -326,46 +327,62 @@ cudaError_t launch_rowpair(const RowPairMaps& maps, const RowPairParams& p, long
 
 }  // namespace
 
-cudaError_t launch_ffn_rowpair_sm100(const moe_config& c, const FfnArgs& f, cudaStream_t s,
-                                     cudaEvent_t mid) {
-  if (c.d % BN != 0 || c.d_ff % (BN / 2) != 0) return cudaErrorInvalidValue;
+static bool rowpair_fits(const moe_config& c) { return c.d % BN == 0 && c.d_ff % (BN / 2) == 0; }
+
+cudaError_t launch_rowpair_gate_up(const moe_config& c, const FfnArgs& f, cudaStream_t s,
+                                   bool routed, bool shared) {
+  if (!rowpair_fits(c)) return cudaErrorInvalidValue;
+  const int nseg = c.E + (c.has_shared ? 1 : 0);
+  const long long rows = (routed ? f.rmax : 0) + (c.has_shared && shared ? c.T : 0);
+  const long long mt_bound = (rows + 2 * BM - 1) / (2 * BM) + nseg;
+  // A = packed rows [rmax, d] (x [T, d] for the shared expert)
+  RowPairMaps m;
+  bool ok = encode_2d_box(&m.a_routed, f.x_packed, c.d, f.rmax, BM) &&
+            encode_2d_box(&m.b0_routed, f.w_gate, c.d, static_cast<uint64_t>(c.E) * c.d_ff, BN / 2) &&
+            encode_2d_box(&m.b1_routed, f.w_up, c.d, static_cast<uint64_t>(c.E) * c.d_ff, BN / 2);
+  if (c.has_shared)
+    ok = ok && encode_2d_box(&m.a_shared, f.x, c.d, c.T, BM) &&
+         encode_2d_box(&m.b0_shared, f.s_gate, c.d, c.d_ff, BN / 2) &&
+         encode_2d_box(&m.b1_shared, f.s_up, c.d, c.d_ff, BN / 2);
+  else
+    m.a_shared = m.a_routed, m.b0_shared = m.b0_routed, m.b1_shared = m.b1_routed;
+  if (!ok) return cudaErrorInvalidValue;
+  RowPairParams p{f.offsets, f.counts, nseg, c.E, c.d, c.d_ff, static_cast<__nv_bfloat16*>(f.h),
+                  c.d_ff, f.status, kWaitLimitNs, routed ? 1 : 0, shared ? 1 : 0};
+  return launch_rowpair<0>(m, p, mt_bound * (c.d_ff / (BN / 2)), s);
+}
+
+cudaError_t launch_rowpair_down(const moe_config& c, const FfnArgs& f, cudaStream_t s,
+                                bool routed, bool shared) {
+  if (!rowpair_fits(c)) return cudaErrorInvalidValue;
   const int nseg = c.E + (c.has_shared ? 1 : 0);
   const long long rows_h = f.rmax + (c.has_shared ? c.T : 0);
-  const long long mt_bound = (rows_h + 2 * BM - 1) / (2 * BM) + nseg;
-
-  // gate/up + SwiGLU:  A = packed rows [rmax, d] (x [T, d] for the shared expert)
-  RowPairMaps m1;
-  bool ok = encode_2d_box(&m1.a_routed, f.x_packed, c.d, f.rmax, BM) &&
-            encode_2d_box(&m1.b0_routed, f.w_gate, c.d, static_cast<uint64_t>(c.E) * c.d_ff, BN / 2) &&
-            encode_2d_box(&m1.b1_routed, f.w_up, c.d, static_cast<uint64_t>(c.E) * c.d_ff, BN / 2);
+  const long long rows = (routed ? f.rmax : 0) + (c.has_shared && shared ? c.T : 0);
+  const long long mt_bound = (rows + 2 * BM - 1) / (2 * BM) + nseg;
+  // A = H [rows_h, F]
+  RowPairMaps m;
+  bool ok = encode_2d_box(&m.a_routed, f.h, c.d_ff, rows_h, BM) &&
+            encode_2d_box(&m.b0_routed, f.w_down, c.d_ff, static_cast<uint64_t>(c.E) * c.d, BN / 2);
   if (c.has_shared)
-    ok = ok && encode_2d_box(&m1.a_shared, f.x, c.d, c.T, BM) &&
-         encode_2d_box(&m1.b0_shared, f.s_gate, c.d, c.d_ff, BN / 2) &&
-         encode_2d_box(&m1.b1_shared, f.s_up, c.d, c.d_ff, BN / 2);
+    ok = ok && encode_2d_box(&m.b0_shared, f.s_down, c.d_ff, c.d, BN / 2);
   else
-    m1.a_shared = m1.a_routed, m1.b0_shared = m1.b0_routed, m1.b1_shared = m1.b1_routed;
+    m.b0_shared = m.b0_routed;
+  m.a_shared = m.a_routed;
+  m.b1_routed = m.b0_routed;
+  m.b1_shared = m.b0_shared;
   if (!ok) return cudaErrorInvalidValue;
-  RowPairParams p1{f.offsets, f.counts, nseg, c.E, c.d, c.d_ff, static_cast<__nv_bfloat16*>(f.h),
-                   c.d_ff, f.status, kWaitLimitNs};
-  cudaError_t e = launch_rowpair<0>(m1, p1, mt_bound * (c.d_ff / (BN / 2)), s);
+  RowPairParams p{f.offsets, f.counts, nseg, c.E, c.d_ff, c.d,
+                  static_cast<__nv_bfloat16*>(f.y_packed), c.d, f.status, kWaitLimitNs,
+                  routed ? 1 : 0, shared ? 1 : 0};
+  return launch_rowpair<1>(m, p, mt_bound * (c.d / BN), s);
+}
+
+cudaError_t launch_ffn_rowpair_sm100(const moe_config& c, const FfnArgs& f, cudaStream_t s,
+                                     cudaEvent_t mid) {
+  cudaError_t e = launch_rowpair_gate_up(c, f, s, true, true);
   if (e != cudaSuccess) return e;
   if (mid != nullptr && (e = record_event(mid, s)) != cudaSuccess) return e;
-
-  // down:  A = H [rows_h, F]
-  RowPairMaps m2;
-  ok = encode_2d_box(&m2.a_routed, f.h, c.d_ff, rows_h, BM) &&
-       encode_2d_box(&m2.b0_routed, f.w_down, c.d_ff, static_cast<uint64_t>(c.E) * c.d, BN / 2);
-  if (c.has_shared)
-    ok = ok && encode_2d_box(&m2.b0_shared, f.s_down, c.d_ff, c.d, BN / 2);
-  else
-    m2.b0_shared = m2.b0_routed;
-  m2.a_shared = m2.a_routed;
-  m2.b1_routed = m2.b0_routed;
-  m2.b1_shared = m2.b0_shared;
-  if (!ok) return cudaErrorInvalidValue;
-  RowPairParams p2{f.offsets, f.counts, nseg, c.E, c.d_ff, c.d,
-                   static_cast<__nv_bfloat16*>(f.y_packed), c.d, f.status, kWaitLimitNs};
-  return launch_rowpair<1>(m2, p2, mt_bound * (c.d / BN), s);
+  return launch_rowpair_down(c, f, s, true, true);
 }
 
 }  // namespace moe

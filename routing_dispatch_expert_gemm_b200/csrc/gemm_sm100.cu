@@ -89,6 +89,7 @@ struct Params {
   int ldo;
   int32_t* status;
   int64_t limit_ns;
+  int routed, shared;      // which segments this launch runs (see build_segment_table)
 };
 
 template <int MODE, int BN>  // MODE 0: SwiGLU gate|up (BN = 256); MODE 1: plain (128/256)
@@ -148,7 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_wait();  // offsets, A rows and the output buffer belong to earlier kernels
   if (warp == 0)  // segment table: row starts and exclusive prefix of tile counts
     gemm::build_segment_table(p.offsets, p.counts, p.nseg, p.E, BM, n_blocks, s_pre, s_row0,
-                              s_rows);
+                              s_rows, p.routed != 0, p.shared != 0);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -371,6 +372,7 @@ int sm_count() {
 // pair tile would be padding (the 64+1 layer at T = 4096, ~128 rows: +16%; decode: +13%;
 // the Granite-shaped layer, ~353 rows: +6%).
 bool row_pairs_fit(const moe_config& c) { return c.d % 256 == 0 && c.d_ff % 128 == 0; }
+constexpr int64_t kPairRows = 512;  // average segment rows from which pairs pay
 
 int32_t ffn_tile_shape(const moe_config& c) {
   if (c.fuse != 0) return MOE_TILES_COLUMNS;  // the fused steps live in the column kernel
@@ -382,10 +384,21 @@ int32_t ffn_tile_shape(const moe_config& c) {
     int64_t rows = static_cast<int64_t>(c.T) * c.k / c.E;
     if (c.capacity >= 0)
       rows = (c.layout == MOE_LAYOUT_PADDED) ? c.capacity : std::min<int64_t>(rows, c.capacity);
-    if (rows >= 512) return MOE_TILES_ROW_PAIRS;
+    if (rows >= kPairRows) return MOE_TILES_ROW_PAIRS;
   }
   return MOE_TILES_ROWS;
 }
+
+// With the automatic choice on row tiles, a shared expert of at least kPairRows rows (its
+// segment is all T tokens) still runs on row tiles over SM pairs, in launches of its own
+// before the routed segments' row tiles (the 64+1 layer at T = 4096: 14.38 -> 13.58 ms per
+// layer on average over three alternating runs; at phi = 1 with reroute -2.4%).
+bool ffn_shared_on_pairs(const moe_config& c) {
+  return c.dtype == MOE_BF16 && c.has_shared && c.T >= kPairRows && c.tiles == MOE_TILES_AUTO &&
+         c.fuse == 0 && row_pairs_fit(c) && ffn_tile_shape(c) == MOE_TILES_ROWS;
+}
+
+int ffn_launches(const moe_config& c) { return ffn_shared_on_pairs(c) ? 4 : 2; }
 
 cudaError_t launch_ffn_sm100(const moe_config& c, const FfnArgs& f, cudaStream_t s,
                              cudaEvent_t mid) {
@@ -395,7 +408,8 @@ cudaError_t launch_ffn_sm100(const moe_config& c, const FfnArgs& f, cudaStream_t
   if (shape == MOE_TILES_ROW_PAIRS) return launch_ffn_rowpair_sm100(c, f, s, mid);
   const int nseg = c.E + (c.has_shared ? 1 : 0);
   const long long rows_h = f.rmax + (c.has_shared ? c.T : 0);
-  const long long mt_bound = (rows_h + BM - 1) / BM + nseg;
+  const bool split = ffn_shared_on_pairs(c);  // the shared segment on row tiles over SM pairs
+  const long long mt_bound = ((split ? f.rmax : rows_h) + BM - 1) / BM + nseg;
 
   // gate/up + SwiGLU:  A = packed rows [rmax, d] (x [T, d] for the shared expert)
   Maps m1;
@@ -409,8 +423,10 @@ cudaError_t launch_ffn_sm100(const moe_config& c, const FfnArgs& f, cudaStream_t
     m1.a_shared = m1.a_routed, m1.b0_shared = m1.b0_routed, m1.b1_shared = m1.b1_routed;
   if (!ok) return cudaErrorInvalidValue;
   Params p1{f.offsets, f.counts, nseg, c.E, c.d, c.d_ff, static_cast<__nv_bfloat16*>(f.h), c.d_ff,
-            f.status, kWaitLimitNs};
-  cudaError_t e = launch_gemm<0, 256>(m1, p1, mt_bound * (c.d_ff / 128), s);
+            f.status, kWaitLimitNs, 1, split ? 0 : 1};
+  cudaError_t e;
+  if (split && (e = launch_rowpair_gate_up(c, f, s, false, true)) != cudaSuccess) return e;
+  e = launch_gemm<0, 256>(m1, p1, mt_bound * (c.d_ff / 128), s);
   if (e != cudaSuccess) return e;
   if (mid != nullptr && (e = record_event(mid, s)) != cudaSuccess) return e;
 
@@ -427,7 +443,8 @@ cudaError_t launch_ffn_sm100(const moe_config& c, const FfnArgs& f, cudaStream_t
   m2.b1_shared = m2.b0_shared;
   if (!ok) return cudaErrorInvalidValue;
   Params p2{f.offsets, f.counts, nseg, c.E, c.d_ff, c.d, static_cast<__nv_bfloat16*>(f.y_packed),
-            c.d, f.status, kWaitLimitNs};
+            c.d, f.status, kWaitLimitNs, 1, split ? 0 : 1};
+  if (split && (e = launch_rowpair_down(c, f, s, false, true)) != cudaSuccess) return e;
   if (c.d % 256 == 0) return launch_gemm<1, 256>(m2, p2, mt_bound * (c.d / 256), s);
   return launch_gemm<1, 128>(m2, p2, mt_bound * (c.d / 128), s);
 }

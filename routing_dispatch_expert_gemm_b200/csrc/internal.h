@@ -157,6 +157,16 @@ cudaError_t launch_ffn_pair_sm100(const moe_config& c, const FfnArgs& a, cudaStr
 // Row tiles over SM pairs (gemm_rowpair_sm100.cu); d a multiple of 256, d_ff of 128.
 cudaError_t launch_ffn_rowpair_sm100(const moe_config& c, const FfnArgs& a, cudaStream_t s,
                                      cudaEvent_t mid = nullptr);
+// One of its GEMMs over a subset of the segments: the routed ones and/or the shared expert's.
+cudaError_t launch_rowpair_gate_up(const moe_config& c, const FfnArgs& a, cudaStream_t s,
+                                   bool routed, bool shared);
+cudaError_t launch_rowpair_down(const moe_config& c, const FfnArgs& a, cudaStream_t s,
+                                bool routed, bool shared);
+// Whether the automatic tile choice runs the shared expert's segment on row tiles over SM
+// pairs, in launches of its own, next to row tiles for the routed segments.
+bool ffn_shared_on_pairs(const moe_config& c);
+// Kernel launches of the expert FFN for the config: 2, or 4 with ffn_shared_on_pairs.
+int ffn_launches(const moe_config& c);
 
 cudaError_t launch_debug_wait(int32_t* status, int64_t limit_ns, cudaStream_t s);
 

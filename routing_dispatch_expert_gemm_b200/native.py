@@ -26,7 +26,7 @@ FUSE = {"none": 0, "gather": 1, "combine": 2, "gather+combine": 3}
 
 # Every symbol include/moe.h declares (checked by the CPU test suite).
 EXPORTS = ("moe_capacity", "moe_max_rows", "moe_workspace_bytes", "moe_workspace_init",
-           "moe_ffn_tile_shape",
+           "moe_ffn_tile_shape", "moe_ffn_launches",
            "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_forward_profiled", "moe_get_device_status", "moe_debug_bounded_wait",
            "moe_dispatch_noalloc", "moe_routing_stats", "moe_status_string",
@@ -99,6 +99,7 @@ def lib() -> ctypes.CDLL:
             "moe_workspace_bytes": (ctypes.c_size_t, [_CFG]),
             "moe_workspace_init": (_I32, [_P, _P]),
             "moe_ffn_tile_shape": (_I32, [_CFG]),
+            "moe_ffn_launches": (_I32, [_CFG]),
             "moe_route": (_I32, [_CFG, _P, _P, _P, _P, _P, _P, _P]),
             "moe_dispatch": (_I32, [_CFG] + [_P] * 10),
             "moe_expert_ffn": (_I32, [_CFG] + [_P] * 12 + [_P]),
@@ -168,6 +169,15 @@ def moe_ffn_tile_shape(cfg: MoeConfig) -> str:
     if v == 0:
         raise MoeError(1, "moe_ffn_tile_shape")
     return {1: "rows", 2: "columns", 3: "pairs", 4: "row_pairs"}[v]
+
+
+def moe_ffn_launches(cfg: MoeConfig) -> int:
+    """Kernel launches of the expert FFN for the config (2, or 4 with the shared expert's
+    segment on SM pairs next to row tiles)."""
+    v = lib().moe_ffn_launches(ctypes.byref(cfg))
+    if v == 0:
+        raise MoeError(1, "moe_ffn_launches")
+    return v
 
 
 def moe_workspace_bytes(cfg: MoeConfig) -> int:

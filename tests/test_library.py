@@ -234,7 +234,16 @@ def test_ffn_tile_shape_choice(native):
         assert native.moe_workspace_bytes(mk(64, 64, 4, 2, 128, dtype="f32", fuse=fuse)) == 0
     assert native.moe_workspace_bytes(mk(1412, 1024, 32, 8, 512, fuse="combine")) > \
         native.moe_workspace_bytes(mk(1412, 1024, 32, 8, 512))
+    # the shared expert's segment on SM pairs next to row tiles: 4 FFN launches instead of 2
+    assert native.moe_ffn_launches(mk(4096, 4096, 64, 2, 32768, has_shared=True)) == 4
+    assert native.moe_ffn_launches(mk(1024, 512, 16, 2, 1024, has_shared=True)) == 4
+    assert native.moe_ffn_launches(mk(511, 4096, 64, 2, 32768, has_shared=True)) == 2
+    assert native.moe_ffn_launches(mk(4096, 4096, 64, 2, 32768, has_shared=True,
+                                      tiles="rows")) == 2
+    assert native.moe_ffn_launches(mk(8192, 4096, 8, 2, 14336)) == 2
+    assert native.moe_ffn_launches(mk(64, 64, 4, 2, 128, dtype="f32", has_shared=True)) == 2
     bad = mk(16, 4096, 8, 2, 14336)
     bad.tiles = 5
     assert native.lib().moe_ffn_tile_shape(ctypes.byref(bad)) == 0
+    assert native.lib().moe_ffn_launches(ctypes.byref(bad)) == 0
     assert native.moe_workspace_bytes(bad) == 0
