@@ -177,7 +177,7 @@ def test_layer_parity_on_oracle_routing(name):
 @pytest.mark.parametrize("name", ["granite_layer", "switch_phi125", "switch_phi050", "mixtral_T300",
                                   "mixtral_decode", "shared64_narrow_phi1",
                                   "shared64_narrow_phi2_T1", "shared16_narrow"])
-def test_both_tile_shapes_on_oracle_routing(name, tiles):
+def test_every_tile_shape_on_oracle_routing(name, tiles):
     """The row-tile, column-tile, column-pair and row-pair FFN kernels, forced on the same
     inputs and routing, each against the oracle (segments of 1 to a few thousand rows,
     ragged tails, the shared expert, capacity drops; the Switch-shaped layers' d = 768 runs
