@@ -194,6 +194,23 @@ def test_every_tile_shape_on_oracle_routing(name, tiles):
     assert_close(out["y"], y_ref, wl.dtype, f"{name} {tiles}")
 
 
+def test_shared_expert_on_pairs_matches_row_tiles_bit_for_bit():
+    """With a shared expert of T >= 512 rows the automatic choice runs that segment on row
+    tiles over SM pairs in launches of its own (4 FFN launches); forcing row tiles runs every
+    segment on one-SM row tiles (2 launches).  Both sum each output element over K in the
+    same order, so the outputs are the same bits; and both meet the oracle."""
+    wl = SMALL["shared16_narrow"]
+    assert N.moe_ffn_launches(config_for(wl)) == 4
+    assert N.moe_ffn_launches(config_for(wl, tiles="rows")) == 2
+    wl_, x, p, C, ids_ref, g32, auto = _run_oracle_routing(wl)
+    _, _, _, _, _, _, rows = _run_oracle_routing(wl, tiles="rows")
+    assert auto["status"] == 0 and rows["status"] == 0
+    assert torch.equal(auto["y"].view(torch.int16), rows["y"].view(torch.int16))
+    y_ref, _ = O.moe_layer(x, p, wl.k, wl.gate_mode, C, add_residual=wl.add_residual,
+                           routing=(ids_ref, g32.double().numpy()))
+    assert_close(auto["y"], y_ref, wl.dtype, "shared16_narrow auto")
+
+
 FUSED_CASES = ["tiny_bf16", "granite_layer", "switch_phi050", "mixtral_T300", "mixtral_decode",
                "shared64_narrow_phi1", "shared64_narrow_dropless", "shared64_narrow_phi2_T1"]
 
